@@ -1,0 +1,400 @@
+// C ABI of libhit.so (declared in include/hit.h): host-side argument checks,
+// pass planning and kernel dispatch.  Every check runs before the first CUDA
+// call, so a rejected call launches nothing; no path falls back to the CPU.
+#include <cmath>
+#include <cstdarg>
+#include <cstdio>
+#include <string>
+
+#include "hit.h"
+#include "internal.h"
+#include "kernels.h"
+
+namespace {
+
+thread_local std::string g_last_error;
+
+int fail(int status, const char* fmt, ...) {
+  char buf[512];
+  va_list ap;
+  va_start(ap, fmt);
+  vsnprintf(buf, sizeof buf, fmt, ap);
+  va_end(ap);
+  g_last_error = buf;
+  return status;
+}
+
+int ok() { return HIT_OK; }
+
+int cuda_status(cudaError_t e, const char* what) {
+  if (e == cudaSuccess) return HIT_OK;
+  return fail(HIT_ECUDA, "%s: %s", what, cudaGetErrorString(e));
+}
+
+bool is_pow2(int64_t v) { return v >= 1 && (v & (v - 1)) == 0; }
+int ilog2(int64_t v) {
+  int k = 0;
+  while ((int64_t(1) << k) < v) ++k;
+  return k;
+}
+size_t esize(int dt) { return dt == HIT_F32 ? 4 : 2; }
+bool dtype_ok(int dt) { return dt == HIT_F32 || dt == HIT_BF16; }
+bool aligned(const void* p, size_t a) { return (reinterpret_cast<uintptr_t>(p) % a) == 0; }
+float inv_sqrt(int64_t n) { return static_cast<float>(1.0 / std::sqrt(static_cast<double>(n))); }
+
+// Row alignment the vector accesses of a row kernel need.
+size_t row_align(int dt, int64_t n) {
+  const int64_t bytes = n * static_cast<int64_t>(esize(dt));
+  return bytes >= 16 ? 16 : static_cast<size_t>(bytes);
+}
+
+int check_rows_operand(const void* p, int64_t ld, int64_t n, int dt, const char* name) {
+  if (p == nullptr) return fail(HIT_EINVAL, "%s is NULL", name);
+  if (ld < n) return fail(HIT_EINVAL, "%s: leading dimension %lld < n %lld", name, (long long)ld, (long long)n);
+  const size_t ra = row_align(dt, n);
+  if (!aligned(p, ra) || (static_cast<size_t>(ld) * esize(dt)) % ra != 0)
+    return fail(HIT_EALIGN, "%s: base and row pitch must be %zu-byte aligned", name, ra);
+  return HIT_OK;
+}
+
+// Column transform of length m on an [m, cols] matrix: ceil(log2(m)/7) passes.
+// tmp (fp32, leading dim ld_tmp) carries the intermediate between passes; it
+// may alias dst when dst is fp32.
+int run_cols(const void* src, int dt_src, int64_t ld_src, void* dst, int dt_dst, int64_t ld_dst, int64_t m,
+             int64_t cols, const int8_t* pre, const int8_t* post, float* tmp, int64_t ld_tmp, cudaStream_t st) {
+  const int k = ilog2(m);
+  const int np = k == 0 ? 1 : (k + 6) / 7;
+  int lo = 0;
+  for (int p = 0; p < np; ++p) {
+    const int nb = (k - lo) / (np - p);  // spread the bits evenly, larger passes last
+    hit::ColArgs a;
+    a.m = m;
+    a.cols = cols;
+    a.lo = lo;
+    const bool first = p == 0, last = p == np - 1;
+    const int nbits = last ? k - lo : nb;
+    a.x = first ? src : tmp;
+    a.ldx = first ? ld_src : ld_tmp;
+    a.y = last ? dst : tmp;
+    a.ldy = last ? ld_dst : ld_tmp;
+    a.pre_signs = first ? pre : nullptr;
+    a.post_signs = last ? post : nullptr;
+    a.norm = last ? inv_sqrt(m) : 1.0f;
+    const cudaError_t e = hit::launch_cols_pass(nbits, first ? dt_src : hit::DT_F32, last ? dt_dst : hit::DT_F32, a, st);
+    if (e != cudaSuccess) return cuda_status(e, "column transform launch");
+    lo += nbits;
+  }
+  return HIT_OK;
+}
+
+int rht_impl(bool inverse, const void* x, void* y, int64_t rows, int64_t n, int64_t ldx, int64_t ldy, int dt_in,
+             int dt_out, const int8_t* signs, int axis, void* ws, size_t ws_bytes, void* stream) {
+  const char* fn = inverse ? "rht_inverse" : "rht_forward";
+  if (!dtype_ok(dt_in) || !dtype_ok(dt_out)) return fail(HIT_EUNSUPPORTED, "%s: unknown dtype", fn);
+  if (rows < 0 || n < 1) return fail(HIT_EINVAL, "%s: bad shape [%lld, %lld]", fn, (long long)rows, (long long)n);
+  if (axis != 0 && axis != 1) return fail(HIT_EINVAL, "%s: axis must be 0 or 1", fn);
+  const int64_t len = axis == 1 ? n : rows;
+  if (!is_pow2(len)) return fail(HIT_EINVAL, "%s: transform length %lld is not a power of two", fn, (long long)len);
+  if (axis == 1 && len > 32768) return fail(HIT_EUNSUPPORTED, "%s: row length %lld > 32768", fn, (long long)len);
+  if (axis == 0 && len > (int64_t(1) << 24)) return fail(HIT_EUNSUPPORTED, "%s: column length > 2^24", fn);
+  int r = check_rows_operand(x, ldx, n, dt_in, "x");
+  if (r) return r;
+  r = check_rows_operand(y, ldy, n, dt_out, "y");
+  if (r) return r;
+  if (signs != nullptr && len >= 4 && !aligned(signs, 4)) return fail(HIT_EALIGN, "%s: signs must be 4-byte aligned", fn);
+  if (rows == 0) return ok();
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  if (axis == 1) {
+    hit::RowArgs a;
+    a.x = x;
+    a.y = y;
+    a.rows = rows;
+    a.ldx = ldx;
+    a.ldy = ldy;
+    a.pre_signs = inverse ? nullptr : signs;
+    a.post_signs = inverse ? signs : nullptr;
+    a.norm = inv_sqrt(n);
+    const int logn = ilog2(n);
+    const cudaError_t e = dt_in == HIT_F32 ? hit::rows_store_from_f32(logn, dt_out, a, st)
+                                           : hit::rows_store_from_bf16(logn, dt_out, a, st);
+    return cuda_status(e, fn);
+  }
+  // columns
+  const int k = ilog2(rows);
+  float* tmp = nullptr;
+  int64_t ld_tmp = 0;
+  if (k > 7) {
+    if (dt_out == HIT_F32) {
+      tmp = static_cast<float*>(y);
+      ld_tmp = ldy;
+    } else {
+      const size_t need = static_cast<size_t>(rows) * static_cast<size_t>(n) * 4;
+      if (ws == nullptr || ws_bytes < need) return fail(HIT_EWORKSPACE, "%s: needs %zu workspace bytes", fn, need);
+      if (!aligned(ws, 16)) return fail(HIT_EALIGN, "%s: workspace must be 16-byte aligned", fn);
+      tmp = static_cast<float*>(ws);
+      ld_tmp = n;
+    }
+  }
+  return run_cols(x, dt_in, ldx, y, dt_out, ldy, rows, n, inverse ? nullptr : signs, inverse ? signs : nullptr, tmp,
+                  ld_tmp, st);
+}
+
+}  // namespace
+
+extern "C" {
+
+int hit_version(void) { return 100; }
+
+const char* hit_status_string(int status) {
+  switch (status) {
+    case HIT_OK: return "ok";
+    case HIT_EINVAL: return "invalid argument";
+    case HIT_EUNSUPPORTED: return "unsupported dtype or size";
+    case HIT_EALIGN: return "misaligned pointer or leading dimension";
+    case HIT_ECUDA: return "CUDA error";
+    case HIT_EWORKSPACE: return "workspace missing or too small";
+  }
+  return "unknown status";
+}
+
+const char* hit_last_error(void) { return g_last_error.c_str(); }
+
+size_t hit_workspace_bytes(int op, int64_t rows, int64_t n, int dtype_out, int flags) {
+  if (rows <= 0 || n <= 0) return 0;
+  const size_t full = static_cast<size_t>(rows) * static_cast<size_t>(n) * 4;
+  switch (op) {
+    case HIT_OP_RHT: return (flags == 0 && rows > 128 && dtype_out != HIT_F32) ? full : 0;
+    case HIT_OP_QUANT: return flags ? full : 0;
+    case HIT_OP_DEQUANT: return (flags && dtype_out != HIT_F32) ? full : 0;
+    case HIT_OP_BUTTERFLY: return (flags > 1 && dtype_out != HIT_F32) ? full : 0;
+  }
+  return 0;
+}
+
+int rht_forward(const void* x, void* y, int64_t rows, int64_t n, int64_t ldx, int64_t ldy, int dtype_in,
+                int dtype_out, const int8_t* signs, int axis, void* workspace, size_t workspace_bytes,
+                void* stream) {
+  return rht_impl(false, x, y, rows, n, ldx, ldy, dtype_in, dtype_out, signs, axis, workspace, workspace_bytes,
+                  stream);
+}
+
+int rht_inverse(const void* x, void* y, int64_t rows, int64_t n, int64_t ldx, int64_t ldy, int dtype_in,
+                int dtype_out, const int8_t* signs, int axis, void* workspace, size_t workspace_bytes,
+                void* stream) {
+  return rht_impl(true, x, y, rows, n, ldx, ldy, dtype_in, dtype_out, signs, axis, workspace, workspace_bytes,
+                  stream);
+}
+
+int butterfly_apply(const void* x, void* y, int64_t rows, int64_t n, int64_t ldx, int64_t ldy, int dtype_in,
+                    int dtype_out, int n_stages, const int32_t* radices, const float* const* blocks,
+                    const int64_t* n_groups, int transpose, int axis, void* workspace, size_t workspace_bytes,
+                    void* stream) {
+  const char* fn = "butterfly_apply";
+  if (!dtype_ok(dtype_in) || !dtype_ok(dtype_out)) return fail(HIT_EUNSUPPORTED, "%s: unknown dtype", fn);
+  if (rows < 0 || n < 1) return fail(HIT_EINVAL, "%s: bad shape", fn);
+  if (axis != 0 && axis != 1) return fail(HIT_EINVAL, "%s: axis must be 0 or 1", fn);
+  if (n_stages < 1 || n_stages > 16) return fail(HIT_EINVAL, "%s: n_stages must be 1..16", fn);
+  if (radices == nullptr || blocks == nullptr || n_groups == nullptr)
+    return fail(HIT_EINVAL, "%s: radices, blocks and n_groups are required", fn);
+  if (x == nullptr || y == nullptr) return fail(HIT_EINVAL, "%s: x and y are required", fn);
+  if (ldx < n || ldy < n) return fail(HIT_EINVAL, "%s: leading dimension < n", fn);
+  if (!aligned(x, esize(dtype_in)) || !aligned(y, esize(dtype_out))) return fail(HIT_EALIGN, "%s: misaligned x or y", fn);
+  const int64_t len = axis == 1 ? n : rows;
+  int64_t prod = 1;
+  for (int t = 0; t < n_stages; ++t) {
+    if (radices[t] < 1 || radices[t] > 64) return fail(HIT_EUNSUPPORTED, "%s: radix %d outside 1..64", fn, radices[t]);
+    prod *= radices[t];
+    if (prod > (int64_t(1) << 40)) return fail(HIT_EINVAL, "%s: radices overflow", fn);
+  }
+  if (prod != len) return fail(HIT_EINVAL, "%s: radices multiply to %lld, transform length is %lld", fn,
+                               (long long)prod, (long long)len);
+  for (int t = 0; t < n_stages; ++t) {
+    if (blocks[t] == nullptr || !aligned(blocks[t], 4)) return fail(HIT_EINVAL, "%s: blocks[%d] missing or misaligned", fn, t);
+    if (n_groups[t] != 1 && n_groups[t] != len / radices[t])
+      return fail(HIT_EINVAL, "%s: n_groups[%d] must be 1 or %lld", fn, t, (long long)(len / radices[t]));
+  }
+  if (rows == 0) return ok();
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  void* tmp = nullptr;
+  int64_t ld_tmp = 0;
+  if (n_stages > 1) {
+    if (dtype_out == HIT_F32) {
+      tmp = y;
+      ld_tmp = ldy;
+    } else {
+      const size_t need = static_cast<size_t>(rows) * static_cast<size_t>(n) * 4;
+      if (workspace == nullptr || workspace_bytes < need) return fail(HIT_EWORKSPACE, "%s: needs %zu workspace bytes", fn, need);
+      if (!aligned(workspace, 16)) return fail(HIT_EALIGN, "%s: workspace must be 16-byte aligned", fn);
+      tmp = workspace;
+      ld_tmp = n;
+    }
+  }
+  for (int p = 0; p < n_stages; ++p) {
+    const int t = transpose ? n_stages - 1 - p : p;
+    int64_t stride = 1;
+    for (int u = t + 1; u < n_stages; ++u) stride *= radices[u];
+    hit::StageArgs a;
+    const bool first = p == 0, last = p == n_stages - 1;
+    a.x = first ? x : tmp;
+    a.ldx = first ? ldx : ld_tmp;
+    a.y = last ? y : tmp;
+    a.ldy = last ? ldy : ld_tmp;
+    a.outer = axis == 1 ? rows : n;
+    a.len = len;
+    a.axis = axis;
+    a.b = radices[t];
+    a.stride = stride;
+    a.blocks = blocks[t];
+    a.shared_block = n_groups[t] == 1 && len / radices[t] != 1 ? 1 : 0;
+    a.transpose = transpose ? 1 : 0;
+    const cudaError_t e = hit::launch_butterfly_stage(first ? dtype_in : HIT_F32, last ? dtype_out : HIT_F32, a, st);
+    if (e != cudaSuccess) return cuda_status(e, fn);
+  }
+  return HIT_OK;
+}
+
+static int check_quant_common(const char* fn, int64_t rows, int64_t n, int bits, int group) {
+  if (rows < 0) return fail(HIT_EINVAL, "%s: rows < 0", fn);
+  if (!is_pow2(n) || n < 32 || n > 32768) return fail(HIT_EUNSUPPORTED, "%s: n must be a power of two in [32, 32768]", fn);
+  if (bits < 2 || bits > 4) return fail(HIT_EUNSUPPORTED, "%s: bits must be 2, 3 or 4", fn);
+  if (!is_pow2(group) || group < 32 || group > n || group > 4096)
+    return fail(HIT_EUNSUPPORTED, "%s: group must be a power of two in [32, min(n, 4096)]", fn);
+  return HIT_OK;
+}
+
+int rht_quantize_pack(const void* x, int64_t rows, int64_t n, int64_t ldx, int dtype_in, const int8_t* row_signs,
+                      const int8_t* col_signs, int bits, int group, uint8_t* codes, float* scales, void* workspace,
+                      size_t workspace_bytes, void* stream) {
+  const char* fn = "rht_quantize_pack";
+  if (!dtype_ok(dtype_in)) return fail(HIT_EUNSUPPORTED, "%s: unknown dtype", fn);
+  int r = check_quant_common(fn, rows, n, bits, group);
+  if (r) return r;
+  r = check_rows_operand(x, ldx, n, dtype_in, "x");
+  if (r) return r;
+  if (codes == nullptr || scales == nullptr) return fail(HIT_EINVAL, "%s: codes and scales are required", fn);
+  if (!aligned(codes, 16) || !aligned(scales, 4)) return fail(HIT_EALIGN, "%s: codes must be 16-byte, scales 4-byte aligned", fn);
+  if ((row_signs && !aligned(row_signs, 4)) || (col_signs && !aligned(col_signs, 4)))
+    return fail(HIT_EALIGN, "%s: signs must be 4-byte aligned", fn);
+  const bool two_sided = col_signs != nullptr;
+  if (two_sided) {
+    if (!is_pow2(rows) || rows > (int64_t(1) << 24)) return fail(HIT_EINVAL, "%s: two-sided needs power-of-two rows", fn);
+    const size_t need = static_cast<size_t>(rows) * static_cast<size_t>(n) * 4;
+    if (workspace == nullptr || workspace_bytes < need) return fail(HIT_EWORKSPACE, "%s: needs %zu workspace bytes", fn, need);
+    if (!aligned(workspace, 16)) return fail(HIT_EALIGN, "%s: workspace must be 16-byte aligned", fn);
+  }
+  if (rows == 0) return ok();
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  hit::RowArgs a;
+  a.rows = rows;
+  a.pre_signs = row_signs;
+  a.norm = inv_sqrt(n);
+  a.codes = codes;
+  a.scales = scales;
+  a.log2g = ilog2(group);
+  int dt_rows = dtype_in;
+  if (two_sided) {
+    float* w = static_cast<float*>(workspace);
+    r = run_cols(x, dtype_in, ldx, w, HIT_F32, n, rows, n, col_signs, nullptr, w, n, st);
+    if (r) return r;
+    a.x = w;
+    a.ldx = n;
+    dt_rows = HIT_F32;
+  } else {
+    a.x = x;
+    a.ldx = ldx;
+  }
+  const int logn = ilog2(n);
+  cudaError_t e;
+  if (bits == 4) e = hit::rows_quant_b4(logn, dt_rows, a, st);
+  else if (bits == 3) e = hit::rows_quant_b3(logn, dt_rows, a, st);
+  else e = hit::rows_quant_b2(logn, dt_rows, a, st);
+  return cuda_status(e, fn);
+}
+
+int dequant_inverse(const uint8_t* codes, const float* scales, int64_t rows, int64_t n, int bits, int group,
+                    const int8_t* row_signs, const int8_t* col_signs, void* y, int64_t ldy, int dtype_out,
+                    void* workspace, size_t workspace_bytes, void* stream) {
+  const char* fn = "dequant_inverse";
+  if (!dtype_ok(dtype_out)) return fail(HIT_EUNSUPPORTED, "%s: unknown dtype", fn);
+  int r = check_quant_common(fn, rows, n, bits, group);
+  if (r) return r;
+  r = check_rows_operand(y, ldy, n, dtype_out, "y");
+  if (r) return r;
+  if (codes == nullptr || scales == nullptr) return fail(HIT_EINVAL, "%s: codes and scales are required", fn);
+  if (!aligned(codes, 16) || !aligned(scales, 4)) return fail(HIT_EALIGN, "%s: codes must be 16-byte, scales 4-byte aligned", fn);
+  if ((row_signs && !aligned(row_signs, 4)) || (col_signs && !aligned(col_signs, 4)))
+    return fail(HIT_EALIGN, "%s: signs must be 4-byte aligned", fn);
+  const bool two_sided = col_signs != nullptr;
+  if (two_sided && (!is_pow2(rows) || rows > (int64_t(1) << 24)))
+    return fail(HIT_EINVAL, "%s: two-sided needs power-of-two rows", fn);
+  if (two_sided && dtype_out != HIT_F32) {
+    const size_t need = static_cast<size_t>(rows) * static_cast<size_t>(n) * 4;
+    if (workspace == nullptr || workspace_bytes < need) return fail(HIT_EWORKSPACE, "%s: needs %zu workspace bytes", fn, need);
+    if (!aligned(workspace, 16)) return fail(HIT_EALIGN, "%s: workspace must be 16-byte aligned", fn);
+  }
+  if (rows == 0) return ok();
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  hit::RowArgs a;
+  a.rows = rows;
+  a.codes_in = codes;
+  a.scales_in = scales;
+  a.log2g = ilog2(group);
+  a.norm = inv_sqrt(n);
+  a.post_signs = row_signs;
+  int dt_rows = dtype_out;
+  float* mid = nullptr;
+  int64_t ld_mid = 0;
+  if (two_sided) {
+    if (dtype_out == HIT_F32) {
+      mid = static_cast<float*>(y);
+      ld_mid = ldy;
+    } else {
+      mid = static_cast<float*>(workspace);
+      ld_mid = n;
+    }
+    a.y = mid;
+    a.ldy = ld_mid;
+    dt_rows = HIT_F32;
+  } else {
+    a.y = y;
+    a.ldy = ldy;
+  }
+  const int logn = ilog2(n);
+  cudaError_t e;
+  if (bits == 4) e = hit::rows_dequant_b4(logn, dt_rows, a, st);
+  else if (bits == 3) e = hit::rows_dequant_b3(logn, dt_rows, a, st);
+  else e = hit::rows_dequant_b2(logn, dt_rows, a, st);
+  r = cuda_status(e, fn);
+  if (r || !two_sided) return r;
+  return run_cols(mid, HIT_F32, ld_mid, y, dtype_out, ldy, rows, n, nullptr, col_signs, mid, ld_mid, st);
+}
+
+int wht_expand_sparse(float* values, const int32_t* cols, int64_t batch, int64_t rows, int64_t n, int32_t nnz,
+                      float scale, float* dense, int mode, void* stream) {
+  const char* fn = "wht_expand_sparse";
+  if (batch < 0 || rows < 0) return fail(HIT_EINVAL, "%s: negative batch or rows", fn);
+  if (!is_pow2(n) || n < 32 || n > 32768) return fail(HIT_EUNSUPPORTED, "%s: n must be a power of two in [32, 32768]", fn);
+  if (nnz < 1 || nnz > n) return fail(HIT_EINVAL, "%s: nnz must be in [1, n]", fn);
+  if (mode != 0 && mode != 1) return fail(HIT_EINVAL, "%s: mode must be 0 or 1", fn);
+  if (values == nullptr || cols == nullptr || dense == nullptr) return fail(HIT_EINVAL, "%s: NULL operand", fn);
+  if (!aligned(values, 4) || !aligned(cols, 4) || !aligned(dense, 16)) return fail(HIT_EALIGN, "%s: misaligned operand", fn);
+  const int64_t total = batch * rows;
+  if (total == 0) return ok();
+  hit::RowArgs a;
+  a.rows = total;
+  a.nnz = nnz;
+  a.sp_cols = cols;
+  a.sp_scale = scale;
+  if (mode == 0) {
+    a.sp_values = values;
+    a.y = dense;
+    a.ldy = n;
+  } else {
+    a.x = dense;
+    a.ldx = n;
+    a.sp_out = values;
+  }
+  return cuda_status(hit::rows_sparse_all(ilog2(n), mode, a, static_cast<cudaStream_t>(stream)), fn);
+}
+
+}  // extern "C"

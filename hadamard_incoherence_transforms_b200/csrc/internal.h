@@ -1,0 +1,75 @@
+// Internal launcher interface between the C ABI (api.cu) and the kernel
+// translation units.  Host-side C++ only; no torch types anywhere.
+#pragma once
+#include <cuda_runtime.h>
+#include <stddef.h>
+#include <stdint.h>
+
+namespace hit {
+
+// Arguments of the row kernels (one CUDA thread team per row; the row length
+// n = 2^logn is a template parameter of the kernel).
+struct RowArgs {
+  const void* x = nullptr;  // dense input rows [rows, ldx]
+  void* y = nullptr;        // dense output rows [rows, ldy]
+  int64_t rows = 0, ldx = 0, ldy = 0;
+  const int8_t* pre_signs = nullptr;   // diag(s) applied on load (forward)
+  const int8_t* post_signs = nullptr;  // diag(s) applied before the store (inverse)
+  float norm = 1.0f;                   // 1/sqrt(n) (or a caller scale)
+  // group quantization (output) / dequantization (input)
+  uint8_t* codes = nullptr;
+  float* scales = nullptr;
+  const uint8_t* codes_in = nullptr;
+  const float* scales_in = nullptr;
+  int log2g = 0;
+  // sparse adapter
+  const float* sp_values = nullptr;
+  const int32_t* sp_cols = nullptr;
+  float* sp_out = nullptr;
+  int nnz = 0;
+  float sp_scale = 1.0f;
+};
+
+// dtype codes (same values as the C ABI)
+enum { DT_F32 = 0, DT_BF16 = 1 };
+
+// y = post(H (pre(x))) * norm along rows, dense in and out.
+cudaError_t launch_rows_store(int logn, int dt_in, int dt_out, const RowArgs& a, cudaStream_t st);
+// Fused transform + group quantization + packing along rows.
+cudaError_t launch_rows_quant(int logn, int dt_in, int bits, const RowArgs& a, cudaStream_t st);
+// Dequantization + inverse transform along rows.
+cudaError_t launch_rows_dequant(int logn, int dt_out, int bits, const RowArgs& a, cudaStream_t st);
+// Sparse adapter: mode 0 scatter + transform, mode 1 transform + gather.
+cudaError_t launch_rows_sparse(int logn, int mode, const RowArgs& a, cudaStream_t st);
+
+// Column (axis 0) transform pass over row-index bits [lo, lo + nb), nb <= 7.
+struct ColArgs {
+  const void* x = nullptr;
+  void* y = nullptr;
+  int64_t m = 0;      // transform length (number of rows), power of two
+  int64_t cols = 0;   // number of columns
+  int64_t ldx = 0, ldy = 0;
+  int lo = 0;         // first row bit of this pass
+  const int8_t* pre_signs = nullptr;
+  const int8_t* post_signs = nullptr;
+  float norm = 1.0f;  // applied on store when != 1
+};
+cudaError_t launch_cols_pass(int nb, int dt_in, int dt_out, const ColArgs& a, cudaStream_t st);
+
+// One mixed-radix butterfly stage (see butterfly_apply in hit.h).
+struct StageArgs {
+  const void* x = nullptr;
+  void* y = nullptr;
+  int64_t outer = 0;        // rows (axis 1) or columns (axis 0)
+  int64_t len = 0;          // transform length
+  int64_t ldx = 0, ldy = 0;
+  int axis = 1;
+  int b = 1;                // radix of this stage
+  int64_t stride = 1;       // S_t = product of the later radices
+  const float* blocks = nullptr;  // [G, b, b]
+  int shared_block = 0;     // 1: one block for all groups
+  int transpose = 0;        // use B^T
+};
+cudaError_t launch_butterfly_stage(int dt_in, int dt_out, const StageArgs& a, cudaStream_t st);
+
+}  // namespace hit

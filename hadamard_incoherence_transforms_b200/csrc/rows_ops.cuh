@@ -1,0 +1,333 @@
+// Epilogues / prologues of the row kernels and the kernels themselves.
+#pragma once
+#include <atomic>
+
+#include "rows.cuh"
+
+namespace hit {
+
+// ----------------------------------------------------------------------------
+// Group-wise symmetric absmax round-to-nearest, in layout B.
+//
+// Per group: a = max|y|, s = a / qmax (IEEE division), q = rint(y / s) with
+// ties to even, stored code u = q + 2^(bits-1).  The division per element is
+// replaced by a multiply with r = 1/s (correctly rounded reciprocal): the
+// exact product y*r differs from the quotient y/s by at most |y/s| * 2^-24 and
+// fl(y/s) from y/s by half an ulp, together < 7e-7 for |y/s| <= qmax <= 7.  So
+// whenever y*r is more than 2^-18 away from a half-integer, fl(y/s) and y*r
+// round to the same integer and the fast result equals rint(fl(y/s)).  A
+// 32-element chunk holding any element inside that margin (probability about
+// 1e-5 per element) is redone with correctly rounded division.  The fast
+// integer comes from fma(y, r, 1.5*2^23 + 2^(bits-1)): that sum lies in
+// [2^23, 2^24) where the float spacing is 1, so its bit pattern is
+// 0x4B400000 + u and the low byte is the stored code.  |y*r| <= a*r <=
+// qmax*(1 + 2^-22) < qmax + 1/2, so the fast path never needs a clamp.
+//
+// When log2(n) is even, 1/sqrt(n) is a power of two and is folded exactly
+// into the scale: y = acc * 2^-k, s = s_acc * 2^-k, y/s = acc/s_acc.
+// ----------------------------------------------------------------------------
+template <int BITS>
+struct QConst {
+  static constexpr float QMAX = float((1 << (BITS - 1)) - 1);
+  static constexpr float MAGIC = 12582912.0f + float(1 << (BITS - 1));
+};
+
+template <int BITS>
+__device__ __forceinline__ void quant_chunk_exact(const float* x, float s, uint32_t* ub) {
+#pragma unroll
+  for (int e = 0; e < 32; ++e) {
+    float q = rintf(__fdiv_rn(x[e], s));
+    q = fminf(fmaxf(q, -QConst<BITS>::QMAX), QConst<BITS>::QMAX);
+    ub[e] = __float_as_uint(q + QConst<BITS>::MAGIC);
+  }
+}
+
+template <int LOGN, int BITS>
+__device__ __forceinline__ void quant_rowB(float (&x)[Geom<LOGN>::E], const RowArgs& a, int64_t row, int tau) {
+  using G = Geom<LOGN>;
+  constexpr int E = G::E;
+  constexpr int NCH = E / 32;
+  constexpr bool FOLD = (LOGN % 2) == 0;
+  constexpr float QMAX = QConst<BITS>::QMAX;
+  constexpr float MAGIC = QConst<BITS>::MAGIC;
+  static_assert(E >= 32, "quantization needs at least 32 elements per thread");
+
+  if constexpr (!FOLD) {
+#pragma unroll
+    for (int e = 0; e < E; e += 2) mul_x2(x[e], x[e + 1], a.norm, a.norm);
+  }
+  float mx[NCH];
+#pragma unroll
+  for (int cc = 0; cc < NCH; ++cc) {
+    float m = 0.0f;
+#pragma unroll
+    for (int e = 0; e < 32; ++e) m = fmaxf(m, fabsf(x[32 * cc + e]));
+    mx[cc] = m;
+  }
+  const int lg = a.log2g;
+#pragma unroll
+  for (int L = 0; (1 << L) < NCH; ++L) {
+    if (5 + L < lg) {
+#pragma unroll
+      for (int cc = 0; cc < NCH; ++cc) {
+        if ((cc >> L) & 1) continue;
+        const float m = fmaxf(mx[cc], mx[cc | (1 << L)]);
+        mx[cc] = m;
+        mx[cc | (1 << L)] = m;
+      }
+    }
+  }
+  if (lg > G::LOGE) {  // a group spans 2^(lg-LOGE) neighbouring threads
+    float m = mx[0];
+    const unsigned mask = team_mask<G::T>();
+    for (int L = 0; L < lg - G::LOGE; ++L) m = fmaxf(m, __shfl_xor_sync(mask, m, 1 << L));
+#pragma unroll
+    for (int cc = 0; cc < NCH; ++cc) mx[cc] = m;
+  }
+
+  constexpr int NW = E * BITS / 32;  // packed words per thread
+  uint32_t W[NW];
+  const int64_t spr = int64_t(G::N) >> lg;
+#pragma unroll
+  for (int cc = 0; cc < NCH; ++cc) {
+    const float s = __fdiv_rn(mx[cc], QMAX);
+    const int e0 = E * tau + 32 * cc;
+    if ((e0 & ((1 << lg) - 1)) == 0) a.scales[row * spr + (e0 >> lg)] = FOLD ? s * a.norm : s;
+    const float* xc = x + 32 * cc;
+    uint32_t ub[32];
+    if (s >= 0x1p-125f) {
+      const float r = __frcp_rn(s);
+      bool risky = false;
+#pragma unroll
+      for (int e = 0; e < 32; ++e) {
+        const float m = fmaf(xc[e], r, MAGIC);
+        const float k = m - MAGIC;
+        const float d = fmaf(xc[e], r, -k);
+        risky |= fabsf(d) > (0.5f - 0x1p-18f);
+        ub[e] = __float_as_uint(m);
+      }
+      if (risky) quant_chunk_exact<BITS>(xc, s, ub);
+    } else if (s > 0.0f) {
+      quant_chunk_exact<BITS>(xc, s, ub);
+    } else {
+#pragma unroll
+      for (int e = 0; e < 32; ++e) ub[e] = __float_as_uint(MAGIC);
+    }
+    if constexpr (BITS == 4) {
+#pragma unroll
+      for (int w = 0; w < 4; ++w) W[4 * cc + w] = pack4x8(ub + 8 * w);
+    } else if constexpr (BITS == 2) {
+#pragma unroll
+      for (int w = 0; w < 2; ++w) W[2 * cc + w] = pack2x16(ub + 16 * w);
+    } else {
+      pack3x32(ub, W + 3 * cc);
+    }
+  }
+  uint8_t* dst = a.codes + row * (int64_t(G::N) * BITS / 8) + int64_t(tau) * (E * BITS / 8);
+  if constexpr (NW % 4 == 0) {
+#pragma unroll
+    for (int v = 0; v < NW / 4; ++v)
+      __stcs(reinterpret_cast<uint4*>(dst) + v, make_uint4(W[4 * v], W[4 * v + 1], W[4 * v + 2], W[4 * v + 3]));
+  } else if constexpr (NW % 2 == 0) {
+#pragma unroll
+    for (int v = 0; v < NW / 2; ++v) __stcs(reinterpret_cast<uint2*>(dst) + v, make_uint2(W[2 * v], W[2 * v + 1]));
+  } else {
+#pragma unroll
+    for (int v = 0; v < NW; ++v) __stcs(reinterpret_cast<uint32_t*>(dst) + v, W[v]);
+  }
+}
+
+// Dequantization into layout B: yhat = (u - 2^(bits-1)) * s, with the
+// transform's 1/sqrt(n) folded into s (exact when log2 n is even).
+template <int LOGN, int BITS>
+__device__ __forceinline__ void dequant_rowB(float (&x)[Geom<LOGN>::E], const RowArgs& a, int64_t row, int tau) {
+  using G = Geom<LOGN>;
+  constexpr int E = G::E;
+  constexpr int NCH = E / 32;
+  constexpr int NW = E * BITS / 32;
+  constexpr float MAGIC = QConst<BITS>::MAGIC;
+  uint32_t W[NW];
+  const uint8_t* src = a.codes_in + row * (int64_t(G::N) * BITS / 8) + int64_t(tau) * (E * BITS / 8);
+  if constexpr (NW % 4 == 0) {
+#pragma unroll
+    for (int v = 0; v < NW / 4; ++v) {
+      const uint4 q = __ldcs(reinterpret_cast<const uint4*>(src) + v);
+      W[4 * v] = q.x;
+      W[4 * v + 1] = q.y;
+      W[4 * v + 2] = q.z;
+      W[4 * v + 3] = q.w;
+    }
+  } else if constexpr (NW % 2 == 0) {
+#pragma unroll
+    for (int v = 0; v < NW / 2; ++v) {
+      const uint2 q = __ldcs(reinterpret_cast<const uint2*>(src) + v);
+      W[2 * v] = q.x;
+      W[2 * v + 1] = q.y;
+    }
+  } else {
+#pragma unroll
+    for (int v = 0; v < NW; ++v) W[v] = __ldcs(reinterpret_cast<const uint32_t*>(src) + v);
+  }
+  const int lg = a.log2g;
+  const int64_t spr = int64_t(G::N) >> lg;
+#pragma unroll
+  for (int cc = 0; cc < NCH; ++cc) {
+    const float s = __ldg(a.scales_in + row * spr + ((E * tau + 32 * cc) >> lg)) * a.norm;
+#pragma unroll
+    for (int e = 0; e < 32; e += 2) {
+      float q0 = __uint_as_float(0x4B400000u | code_at<BITS>(W + BITS * cc, e)) - MAGIC;
+      float q1 = __uint_as_float(0x4B400000u | code_at<BITS>(W + BITS * cc, e + 1)) - MAGIC;
+      mul_x2(q0, q1, s, s);
+      x[32 * cc + e] = q0;
+      x[32 * cc + e + 1] = q1;
+    }
+  }
+}
+
+// Sparse adapter, forward: F_r = scatter-add of (values * scale) at cols into
+// a zeroed row buffer, then read back in layout B.
+template <int LOGN>
+__device__ __forceinline__ void scatter_rowB(float (&x)[Geom<LOGN>::E], const RowArgs& a, int64_t row, int tau,
+                                             int team, float4* buf) {
+  using G = Geom<LOGN>;
+#pragma unroll
+  for (int m = 0; m < G::E / 4; ++m) buf[swz<G::LQ>((G::E / 4) * tau + m)] = make_float4(0.f, 0.f, 0.f, 0.f);
+  team_sync<G::T>(team);
+  float* bf = reinterpret_cast<float*>(buf);
+  const int64_t base = row * a.nnz;
+  for (int k = tau; k < a.nnz; k += G::T) {
+    const int col = __ldg(a.sp_cols + base + k);
+    if (static_cast<unsigned>(col) < static_cast<unsigned>(G::N))
+      atomicAdd(bf + smem_elem<LOGN>(col), __ldg(a.sp_values + base + k) * a.sp_scale);
+  }
+  team_sync<G::T>(team);
+  smem_get_B<LOGN>(buf, x, tau);
+}
+
+// Sparse adapter, backward: out[k] = (row transform * scale)[cols[k]].
+template <int LOGN>
+__device__ __forceinline__ void gather_rowB(const float (&x)[Geom<LOGN>::E], const RowArgs& a, int64_t row, int tau,
+                                            int team, float4* buf) {
+  using G = Geom<LOGN>;
+  smem_put_B<LOGN>(buf, x, tau);
+  team_sync<G::T>(team);
+  const float* bf = reinterpret_cast<const float*>(buf);
+  const int64_t base = row * a.nnz;
+  for (int k = tau; k < a.nnz; k += G::T) {
+    const int col = __ldg(a.sp_cols + base + k);
+    float v = 0.0f;
+    if (static_cast<unsigned>(col) < static_cast<unsigned>(G::N)) v = bf[smem_elem<LOGN>(col)] * a.sp_scale;
+    a.sp_out[base + k] = v;
+  }
+}
+
+enum { EPI_STORE = 0, EPI_QUANT = 1, EPI_GATHER = 2 };
+enum { PRO_DEQUANT = 0, PRO_SCATTER = 1 };
+
+// Dense rows in (layout A), transform, result in layout B.
+template <int LOGN, typename Tin, typename Tout, int EPI, int BITS>
+__global__ void __launch_bounds__(Geom<LOGN>::NT, Geom<LOGN>::MINB) k_rows_a2b(const RowArgs a) {
+  using G = Geom<LOGN>;
+  extern __shared__ float4 smem4[];
+  const int tid = threadIdx.x;
+  const int team = tid >> G::LOGT;
+  const int tau = tid & (G::T - 1);
+  const int64_t row = int64_t(blockIdx.x) * G::RPC + team;
+  if (row >= a.rows) return;  // whole teams leave together
+  float4* buf = smem4 + size_t(team) * (G::N / 4);
+
+  float x[G::E];
+  load_rowA<LOGN, Tin>(x, static_cast<const Tin*>(a.x) + row * a.ldx, tau, a.pre_signs);
+  reg_stages<G::E, 0, G::LOGE>(x);
+  if constexpr (G::T > 1) {
+    smem_put_A<LOGN>(buf, x, tau);
+    team_sync<G::T>(team);
+    smem_get_B<LOGN>(buf, x, tau);
+    reg_stages<G::E, 2, G::B_FWD_HI>(x);
+#pragma unroll
+    for (int b = 0; b < G::NSH; ++b) shfl_stage<G::E>(x, b, (tau >> b) & 1);
+  }
+  if constexpr (EPI == EPI_STORE) {
+    store_rowB<LOGN, Tout>(x, static_cast<Tout*>(a.y) + row * a.ldy, tau, a.norm, a.post_signs);
+  } else if constexpr (EPI == EPI_QUANT) {
+    quant_rowB<LOGN, BITS>(x, a, row, tau);
+  } else {
+    gather_rowB<LOGN>(x, a, row, tau, team, buf);
+  }
+}
+
+// Rows produced in layout B (dequantized codes or a scattered sparse row),
+// transform, dense result stored in layout A.
+template <int LOGN, typename Tout, int PRO, int BITS>
+__global__ void __launch_bounds__(Geom<LOGN>::NT, Geom<LOGN>::MINB) k_rows_b2a(const RowArgs a) {
+  using G = Geom<LOGN>;
+  extern __shared__ float4 smem4[];
+  const int tid = threadIdx.x;
+  const int team = tid >> G::LOGT;
+  const int tau = tid & (G::T - 1);
+  const int64_t row = int64_t(blockIdx.x) * G::RPC + team;
+  if (row >= a.rows) return;
+  float4* buf = smem4 + size_t(team) * (G::N / 4);
+
+  float x[G::E];
+  if constexpr (PRO == PRO_DEQUANT) {
+    dequant_rowB<LOGN, BITS>(x, a, row, tau);
+  } else {
+    scatter_rowB<LOGN>(x, a, row, tau, team, buf);
+  }
+  reg_stages<G::E, 0, G::LOGE>(x);
+  if constexpr (G::T > 1) {
+#pragma unroll
+    for (int b = 0; b < G::NSH; ++b) shfl_stage<G::E>(x, b, (tau >> b) & 1);
+    smem_put_B<LOGN>(buf, x, tau);
+    team_sync<G::T>(team);
+    smem_get_A<LOGN>(buf, x, tau);
+    reg_stages<G::E, G::A_INV_LO, G::LOGE>(x);
+  }
+  store_rowA<LOGN, Tout, false>(x, static_cast<Tout*>(a.y) + row * a.ldy, tau, 1.0f, a.post_signs);
+}
+
+// ----------------------------------------------------------------------------
+// Host launch helpers.
+// ----------------------------------------------------------------------------
+// Opt a kernel into more than 48 KB of dynamic shared memory, once per device.
+template <typename K>
+inline cudaError_t set_smem_attr(K kernel, size_t smem, std::atomic<unsigned long long>& done_mask) {
+  if (smem <= 48 * 1024) return cudaSuccess;
+  int dev = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return e;
+  const unsigned long long bit = 1ull << (dev & 63);
+  if (done_mask.load(std::memory_order_acquire) & bit) return cudaSuccess;
+  e = cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, int(smem));
+  if (e == cudaSuccess) done_mask.fetch_or(bit, std::memory_order_acq_rel);
+  return e;
+}
+
+template <int LOGN, typename Tin, typename Tout, int EPI, int BITS>
+cudaError_t launch_a2b(const RowArgs& a, cudaStream_t st) {
+  using G = Geom<LOGN>;
+  static std::atomic<unsigned long long> done{0};
+  auto kern = k_rows_a2b<LOGN, Tin, Tout, EPI, BITS>;
+  const size_t smem = G::smem_bytes(EPI == EPI_GATHER);
+  cudaError_t e = set_smem_attr(kern, smem, done);
+  if (e != cudaSuccess) return e;
+  const int64_t grid = (a.rows + G::RPC - 1) / G::RPC;
+  kern<<<dim3(unsigned(grid)), G::NT, smem, st>>>(a);
+  return cudaGetLastError();
+}
+
+template <int LOGN, typename Tout, int PRO, int BITS>
+cudaError_t launch_b2a(const RowArgs& a, cudaStream_t st) {
+  using G = Geom<LOGN>;
+  static std::atomic<unsigned long long> done{0};
+  auto kern = k_rows_b2a<LOGN, Tout, PRO, BITS>;
+  const size_t smem = G::smem_bytes(PRO == PRO_SCATTER);
+  cudaError_t e = set_smem_attr(kern, smem, done);
+  if (e != cudaSuccess) return e;
+  const int64_t grid = (a.rows + G::RPC - 1) / G::RPC;
+  kern<<<dim3(unsigned(grid)), G::NT, smem, st>>>(a);
+  return cudaGetLastError();
+}
+
+}  // namespace hit

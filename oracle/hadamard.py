@@ -93,3 +93,55 @@ def two_sided(w, row_signs, col_signs) -> np.ndarray:
 def two_sided_inverse(wp, row_signs, col_signs) -> np.ndarray:
     """Inverse of :func:`two_sided`."""
     return irht_rows(irht_cols(wp, col_signs), row_signs)
+
+
+def hadamard_rows(n: int, idx) -> np.ndarray:
+    """Selected rows of H_n from the entry formula H[i, j] = (-1)^popcount(i & j)
+    (the closed form of the Sylvester recursion; H is symmetric, so these are
+    also its columns).  Used to evaluate sampled outputs of large transforms."""
+    if not is_pow2(n):
+        raise ValueError(f"n={n} is not a power of two")
+    i = np.asarray(idx, dtype=np.int64)[:, None]
+    v = i & np.arange(n, dtype=np.int64)[None, :]
+    par = np.zeros(v.shape, dtype=np.int64)
+    while np.any(v):
+        par ^= v & 1
+        v >>= 1
+    return np.where(par == 1, -1.0, 1.0)
+
+
+def rht_rows_at(x, signs, cols) -> np.ndarray:
+    """Columns `cols` of the row-wise forward transform of x (float64)."""
+    x = np.asarray(x, dtype=np.float64)
+    n = x.shape[-1]
+    return ((x * _signs(signs, n)) @ hadamard_rows(n, cols).T) / np.sqrt(n)
+
+
+def two_sided_rows_at(w, row_signs, col_signs, rows_idx) -> np.ndarray:
+    """Rows `rows_idx` of two_sided(w, row_signs, col_signs): the column transform
+    restricted to those output rows, then the full row transform."""
+    w = np.asarray(w, dtype=np.float64)
+    m = w.shape[0]
+    z = ((hadamard_rows(m, rows_idx) * _signs(col_signs, m)) @ w) / np.sqrt(m)
+    return rht_rows(z, row_signs)
+
+
+def two_sided_inverse_rows_at(wp, row_signs, col_signs, rows_idx) -> np.ndarray:
+    """Rows `rows_idx` of two_sided_inverse(wp, ...): the inverse column transform
+    restricted to those rows, then the full inverse row transform."""
+    wp = np.asarray(wp, dtype=np.float64)
+    m = wp.shape[0]
+    idx = np.asarray(rows_idx)
+    z = (hadamard_rows(m, idx) @ wp) / np.sqrt(m) * _signs(col_signs, m)[idx][:, None]
+    return irht_rows(z, row_signs)
+
+
+def rht_rows_chunked(x, signs, chunk: int = 1024) -> np.ndarray:
+    """rht_rows for long rows, building H_n a block of columns at a time."""
+    x = np.asarray(x, dtype=np.float64)
+    n = x.shape[-1]
+    out = np.empty(x.shape, dtype=np.float64)
+    for c0 in range(0, n, chunk):
+        cols = np.arange(c0, min(n, c0 + chunk))
+        out[..., cols] = rht_rows_at(x, signs, cols)
+    return out

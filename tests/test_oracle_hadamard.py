@@ -93,3 +93,32 @@ def test_two_sided_matches_explicit_products(m, n):
     # column transform alone is the left factor
     np.testing.assert_allclose(oh.rht_cols(w, s_out), left @ w, atol=1e-12)
     np.testing.assert_allclose(oh.irht_cols(left @ w, s_out), w, atol=1e-12)
+
+
+@pytest.mark.parametrize("n", [1, 2, 64, 1024])
+def test_hadamard_rows_equal_sylvester(n):
+    idx = np.unique(np.random.default_rng(n).integers(0, n, size=min(n, 17)))
+    assert np.array_equal(oh.hadamard_rows(n, idx), oh.sylvester(n)[idx])
+
+
+def test_sampled_outputs_equal_full_transforms():
+    rng = np.random.default_rng(21)
+    m, n = 64, 256
+    w = rng.standard_normal((m, n))
+    s_in, s_out = rng.choice([-1, 1], n), rng.choice([-1, 1], m)
+    cols = np.array([0, 5, 255])
+    np.testing.assert_allclose(oh.rht_rows_at(w, s_in, cols), oh.rht_rows(w, s_in)[:, cols], atol=1e-12)
+    rows = np.array([1, 30, 63])
+    np.testing.assert_allclose(oh.two_sided_rows_at(w, s_in, s_out, rows), oh.two_sided(w, s_in, s_out)[rows],
+                               atol=1e-12)
+
+
+def test_sampled_inverse_and_chunked_forward():
+    rng = np.random.default_rng(22)
+    m, n = 32, 128
+    wp = rng.standard_normal((m, n))
+    s_in, s_out = rng.choice([-1, 1], n), rng.choice([-1, 1], m)
+    rows = np.array([0, 7, 31])
+    np.testing.assert_allclose(oh.two_sided_inverse_rows_at(wp, s_in, s_out, rows),
+                               oh.two_sided_inverse(wp, s_in, s_out)[rows], atol=1e-12)
+    np.testing.assert_allclose(oh.rht_rows_chunked(wp, s_in, chunk=48), oh.rht_rows(wp, s_in), atol=1e-12)
