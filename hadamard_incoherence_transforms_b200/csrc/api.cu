@@ -48,6 +48,14 @@ size_t row_align(int dt, int64_t n) {
   return bytes >= 16 ? 16 : static_cast<size_t>(bytes);
 }
 
+// Column passes access single elements: only element alignment is needed.
+int check_cols_operand(const void* p, int64_t ld, int64_t n, int dt, const char* name) {
+  if (p == nullptr) return fail(HIT_EINVAL, "%s is NULL", name);
+  if (ld < n) return fail(HIT_EINVAL, "%s: leading dimension %lld < n %lld", name, (long long)ld, (long long)n);
+  if (!aligned(p, esize(dt))) return fail(HIT_EALIGN, "%s: base must be %zu-byte aligned", name, esize(dt));
+  return HIT_OK;
+}
+
 int check_rows_operand(const void* p, int64_t ld, int64_t n, int dt, const char* name) {
   if (p == nullptr) return fail(HIT_EINVAL, "%s is NULL", name);
   if (ld < n) return fail(HIT_EINVAL, "%s: leading dimension %lld < n %lld", name, (long long)ld, (long long)n);
@@ -97,9 +105,9 @@ int rht_impl(bool inverse, const void* x, void* y, int64_t rows, int64_t n, int6
   if (!is_pow2(len)) return fail(HIT_EINVAL, "%s: transform length %lld is not a power of two", fn, (long long)len);
   if (axis == 1 && len > 32768) return fail(HIT_EUNSUPPORTED, "%s: row length %lld > 32768", fn, (long long)len);
   if (axis == 0 && len > (int64_t(1) << 24)) return fail(HIT_EUNSUPPORTED, "%s: column length > 2^24", fn);
-  int r = check_rows_operand(x, ldx, n, dt_in, "x");
+  int r = axis == 1 ? check_rows_operand(x, ldx, n, dt_in, "x") : check_cols_operand(x, ldx, n, dt_in, "x");
   if (r) return r;
-  r = check_rows_operand(y, ldy, n, dt_out, "y");
+  r = axis == 1 ? check_rows_operand(y, ldy, n, dt_out, "y") : check_cols_operand(y, ldy, n, dt_out, "y");
   if (r) return r;
   if (signs != nullptr && len >= 4 && !aligned(signs, 4)) return fail(HIT_EALIGN, "%s: signs must be 4-byte aligned", fn);
   if (rows == 0) return ok();
