@@ -65,6 +65,13 @@ int check_rows_operand(const void* p, int64_t ld, int64_t n, int dt, const char*
   return HIT_OK;
 }
 
+// Rows of 4096 or 8192 elements go through the persistent TMA-fed kernel; its
+// bulk copies need 16-byte aligned row starts (always true for the row
+// pitches the checks accept when n >= 4096).
+bool use_stream(int logn, const void* x, int64_t ld, int dt) {
+  return (logn == 12 || logn == 13) && aligned(x, 16) && (static_cast<size_t>(ld) * esize(dt)) % 16 == 0;
+}
+
 // Column transform of length m on an [m, cols] matrix: ceil(log2(m)/7) passes.
 // tmp (fp32, leading dim ld_tmp) carries the intermediate between passes; it
 // may alias dst when dst is fp32.
@@ -101,6 +108,7 @@ int rht_impl(bool inverse, const void* x, void* y, int64_t rows, int64_t n, int6
   if (!dtype_ok(dt_in) || !dtype_ok(dt_out)) return fail(HIT_EUNSUPPORTED, "%s: unknown dtype", fn);
   if (rows < 0 || n < 1) return fail(HIT_EINVAL, "%s: bad shape [%lld, %lld]", fn, (long long)rows, (long long)n);
   if (axis != 0 && axis != 1) return fail(HIT_EINVAL, "%s: axis must be 0 or 1", fn);
+  if (rows == 0) return ok();  // empty input: nothing to read or write
   const int64_t len = axis == 1 ? n : rows;
   if (!is_pow2(len)) return fail(HIT_EINVAL, "%s: transform length %lld is not a power of two", fn, (long long)len);
   if (axis == 1 && len > 32768) return fail(HIT_EUNSUPPORTED, "%s: row length %lld > 32768", fn, (long long)len);
@@ -123,8 +131,10 @@ int rht_impl(bool inverse, const void* x, void* y, int64_t rows, int64_t n, int6
     a.post_signs = inverse ? signs : nullptr;
     a.norm = inv_sqrt(n);
     const int logn = ilog2(n);
-    const cudaError_t e = dt_in == HIT_F32 ? hit::rows_store_from_f32(logn, dt_out, a, st)
-                                           : hit::rows_store_from_bf16(logn, dt_out, a, st);
+    cudaError_t e;
+    if (use_stream(logn, x, ldx, dt_in)) e = hit::rows_stream_store(logn, dt_in, dt_out, a, st);
+    else if (dt_in == HIT_F32) e = hit::rows_store_from_f32(logn, dt_out, a, st);
+    else e = hit::rows_store_from_bf16(logn, dt_out, a, st);
     return cuda_status(e, fn);
   }
   // columns
@@ -202,6 +212,7 @@ int butterfly_apply(const void* x, void* y, int64_t rows, int64_t n, int64_t ldx
   if (rows < 0 || n < 1) return fail(HIT_EINVAL, "%s: bad shape", fn);
   if (axis != 0 && axis != 1) return fail(HIT_EINVAL, "%s: axis must be 0 or 1", fn);
   if (n_stages < 1 || n_stages > 16) return fail(HIT_EINVAL, "%s: n_stages must be 1..16", fn);
+  if (rows == 0) return ok();
   if (radices == nullptr || blocks == nullptr || n_groups == nullptr)
     return fail(HIT_EINVAL, "%s: radices, blocks and n_groups are required", fn);
   if (x == nullptr || y == nullptr) return fail(HIT_EINVAL, "%s: x and y are required", fn);
@@ -277,6 +288,7 @@ int rht_quantize_pack(const void* x, int64_t rows, int64_t n, int64_t ldx, int d
   if (!dtype_ok(dtype_in)) return fail(HIT_EUNSUPPORTED, "%s: unknown dtype", fn);
   int r = check_quant_common(fn, rows, n, bits, group);
   if (r) return r;
+  if (rows == 0) return ok();
   r = check_rows_operand(x, ldx, n, dtype_in, "x");
   if (r) return r;
   if (codes == nullptr || scales == nullptr) return fail(HIT_EINVAL, "%s: codes and scales are required", fn);
@@ -313,7 +325,8 @@ int rht_quantize_pack(const void* x, int64_t rows, int64_t n, int64_t ldx, int d
   }
   const int logn = ilog2(n);
   cudaError_t e;
-  if (bits == 4) e = hit::rows_quant_b4(logn, dt_rows, a, st);
+  if (use_stream(logn, a.x, a.ldx, dt_rows)) e = hit::rows_stream_quant(logn, dt_rows, bits, a, st);
+  else if (bits == 4) e = hit::rows_quant_b4(logn, dt_rows, a, st);
   else if (bits == 3) e = hit::rows_quant_b3(logn, dt_rows, a, st);
   else e = hit::rows_quant_b2(logn, dt_rows, a, st);
   return cuda_status(e, fn);
@@ -326,6 +339,7 @@ int dequant_inverse(const uint8_t* codes, const float* scales, int64_t rows, int
   if (!dtype_ok(dtype_out)) return fail(HIT_EUNSUPPORTED, "%s: unknown dtype", fn);
   int r = check_quant_common(fn, rows, n, bits, group);
   if (r) return r;
+  if (rows == 0) return ok();
   r = check_rows_operand(y, ldy, n, dtype_out, "y");
   if (r) return r;
   if (codes == nullptr || scales == nullptr) return fail(HIT_EINVAL, "%s: codes and scales are required", fn);
@@ -384,6 +398,7 @@ int wht_expand_sparse(float* values, const int32_t* cols, int64_t batch, int64_t
   if (!is_pow2(n) || n < 32 || n > 32768) return fail(HIT_EUNSUPPORTED, "%s: n must be a power of two in [32, 32768]", fn);
   if (nnz < 1 || nnz > n) return fail(HIT_EINVAL, "%s: nnz must be in [1, n]", fn);
   if (mode != 0 && mode != 1) return fail(HIT_EINVAL, "%s: mode must be 0 or 1", fn);
+  if (batch * rows == 0) return ok();
   if (values == nullptr || cols == nullptr || dense == nullptr) return fail(HIT_EINVAL, "%s: NULL operand", fn);
   if (!aligned(values, 4) || !aligned(cols, 4) || !aligned(dense, 16)) return fail(HIT_EALIGN, "%s: misaligned operand", fn);
   const int64_t total = batch * rows;

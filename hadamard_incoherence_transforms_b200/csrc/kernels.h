@@ -12,4 +12,8 @@ cudaError_t rows_dequant_b2(int logn, int dt_out, const RowArgs& a, cudaStream_t
 cudaError_t rows_dequant_b3(int logn, int dt_out, const RowArgs& a, cudaStream_t st);
 cudaError_t rows_dequant_b4(int logn, int dt_out, const RowArgs& a, cudaStream_t st);
 cudaError_t rows_sparse_all(int logn, int mode, const RowArgs& a, cudaStream_t st);
+// Persistent TMA-fed variants for n = 4096 / 8192.
+cudaError_t rows_stream_quant(int logn, int dt_in, int bits, const RowArgs& a, cudaStream_t st);
+cudaError_t rows_stream_store(int logn, int dt_in, int dt_out, const RowArgs& a, cudaStream_t st);
+unsigned int read_wait_timeouts();
 }  // namespace hit
