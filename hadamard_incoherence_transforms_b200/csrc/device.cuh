@@ -181,9 +181,9 @@ __device__ __forceinline__ uint32_t code_at(const uint32_t* w, int e) {
 
 namespace hit {
 // ---------------------------------------------------------------------------
-// mbarrier + 1-D bulk async copy (TMA) helpers.  Every wait is bounded: it
-// gives up after ~2^24 polls and reports failure to the caller, which records
-// it in a device counter and stops.
+// mbarrier + 1-D bulk async copy (TMA) helpers.  Every wait is bounded in
+// time: it gives up after about two seconds (global timer) and reports
+// failure to the caller, which records it in a device counter and stops.
 // ---------------------------------------------------------------------------
 __device__ __forceinline__ uint32_t smem_u32(const void* p) {
   return static_cast<uint32_t>(__cvta_generic_to_shared(p));
@@ -212,10 +212,19 @@ __device__ __forceinline__ bool mbar_try_wait(uint64_t* bar, uint32_t parity) {
       : "memory");
   return ok != 0;
 }
+__device__ __forceinline__ uint64_t global_ns() {
+  uint64_t t;
+  asm volatile("mov.u64 %0, %%globaltimer;" : "=l"(t));
+  return t;
+}
+// Wait for phase `parity` of an mbarrier; false after about two seconds.
 __device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity) {
-  for (uint32_t i = 0; i < (1u << 24); ++i)
+  if (mbar_try_wait(bar, parity)) return true;
+  const uint64_t t0 = global_ns();
+  for (uint32_t i = 1;; ++i) {
     if (mbar_try_wait(bar, parity)) return true;
-  return false;
+    if ((i & 63) == 0 && global_ns() - t0 > 2000000000ull) return false;
+  }
 }
 // global -> shared bulk copy; dst and src 16-byte aligned, bytes a multiple of 16.
 __device__ __forceinline__ void bulk_g2s(void* dst, const void* src, uint32_t bytes, uint64_t* bar) {
