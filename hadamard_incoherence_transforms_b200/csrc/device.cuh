@@ -43,6 +43,20 @@ __device__ __forceinline__ void mul_x2(float& a0, float& a1, float m0, float m1)
   upk2(R, a0, a1);
 }
 
+// {d0, d1} = {a0, a1} * {b0, b1} + {c0, c1}, one rounding per lane
+__device__ __forceinline__ void fma_x2(float a0, float a1, float b0, float b1, float c0, float c1, float& d0,
+                                       float& d1) {
+  unsigned long long A = pk2(a0, a1), B = pk2(b0, b1), C = pk2(c0, c1), D;
+  asm("fma.rn.f32x2 %0, %1, %2, %3;" : "=l"(D) : "l"(A), "l"(B), "l"(C));
+  upk2(D, d0, d1);
+}
+// {d0, d1} = {a0, a1} - {b0, b1}
+__device__ __forceinline__ void sub_x2(float a0, float a1, float b0, float b1, float& d0, float& d1) {
+  unsigned long long A = pk2(a0, a1), B = pk2(b0, b1), D;
+  asm("sub.rn.f32x2 %0, %1, %2;" : "=l"(D) : "l"(A), "l"(B));
+  upk2(D, d0, d1);
+}
+
 // One Hadamard stage on register-index bit Q of a thread-private array: for
 // every r with bit Q clear, (x[r], x[r + 2^Q]) <- (x[r] + x[r+2^Q], x[r] - x[r+2^Q]).
 template <int E, int Q>

@@ -58,11 +58,13 @@ __device__ __forceinline__ void quant_rowB(float (&x)[Geom<LOGN>::E], const RowA
   }
   float mx[NCH];
 #pragma unroll
-  for (int cc = 0; cc < NCH; ++cc) {
-    float m = 0.0f;
+  for (int cc = 0; cc < NCH; ++cc) {  // |max| over 32 elements as a tree (independent chains)
+    float t[8];
 #pragma unroll
-    for (int e = 0; e < 32; ++e) m = fmaxf(m, fabsf(x[32 * cc + e]));
-    mx[cc] = m;
+    for (int k = 0; k < 8; ++k)
+      t[k] = fmaxf(fmaxf(fabsf(x[32 * cc + k]), fabsf(x[32 * cc + 8 + k])),
+                   fmaxf(fabsf(x[32 * cc + 16 + k]), fabsf(x[32 * cc + 24 + k])));
+    mx[cc] = fmaxf(fmaxf(fmaxf(t[0], t[1]), fmaxf(t[2], t[3])), fmaxf(fmaxf(t[4], t[5]), fmaxf(t[6], t[7])));
   }
   const int lg = a.log2g;
 #pragma unroll
@@ -97,16 +99,19 @@ __device__ __forceinline__ void quant_rowB(float (&x)[Geom<LOGN>::E], const RowA
     uint32_t ub[32];
     if (s >= 0x1p-125f) {
       const float r = __frcp_rn(s);
-      bool risky = false;
+      // m = fl(y*r + MAGIC) (the rounded code), d = fl(y*r - (m - MAGIC)) its residual
+      float dmax = 0.0f;
 #pragma unroll
-      for (int e = 0; e < 32; ++e) {
-        const float m = fmaf(xc[e], r, MAGIC);
-        const float k = m - MAGIC;
-        const float d = fmaf(xc[e], r, -k);
-        risky |= fabsf(d) > (0.5f - 0x1p-18f);
-        ub[e] = __float_as_uint(m);
+      for (int e = 0; e < 32; e += 2) {
+        float m0, m1, n0, n1, d0, d1;
+        fma_x2(xc[e], xc[e + 1], r, r, MAGIC, MAGIC, m0, m1);
+        sub_x2(MAGIC, MAGIC, m0, m1, n0, n1);
+        fma_x2(xc[e], xc[e + 1], r, r, n0, n1, d0, d1);
+        dmax = fmaxf(dmax, fmaxf(fabsf(d0), fabsf(d1)));
+        ub[e] = __float_as_uint(m0);
+        ub[e + 1] = __float_as_uint(m1);
       }
-      if (risky) quant_chunk_exact<BITS>(xc, s, ub);
+      if (dmax > 0.5f - 0x1p-18f) quant_chunk_exact<BITS>(xc, s, ub);
     } else if (s > 0.0f) {
       quant_chunk_exact<BITS>(xc, s, ub);
     } else {

@@ -39,8 +39,9 @@ struct StreamCfg {
   static constexpr int TEAMS = NCW / WPR;                      // rows in compute at once
   static constexpr uint32_t SLOT = uint32_t(G::N) * 4;         // fp32 row (transpose space)
   static constexpr uint32_t ROW = uint32_t(G::N) * sizeof(Tin);
-  static constexpr int S = (HIT_STREAM_RING_BYTES) / SLOT;     // ring depth
-  static constexpr size_t SMEM = 1024 + size_t(S) * SLOT;
+  static constexpr uint32_t SIGNS = uint32_t(G::N) * 4;        // +-1.0 per column
+  static constexpr int S = (HIT_STREAM_RING_BYTES - SIGNS) / SLOT;  // ring depth
+  static constexpr size_t SMEM = 1024 + SIGNS + size_t(S) * SLOT;
   static constexpr int THREADS = (NCW + 1) * 32;
   static_assert(S >= 2, "ring needs at least two slots");
 };
@@ -61,8 +62,13 @@ __global__ void __launch_bounds__(StreamCfg<LOGN, Tin>::THREADS, 1) k_rows_strea
   extern __shared__ __align__(1024) uint8_t smem[];
   uint64_t* full = reinterpret_cast<uint64_t*>(smem);
   uint64_t* empty = full + C::S;
-  uint8_t* slots = smem + 1024;
+  float* sgn = reinterpret_cast<float*>(smem + 1024);
+  uint8_t* slots = smem + 1024 + C::SIGNS;
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const bool has_signs = a.pre_signs != nullptr;
+  if (has_signs) {  // the sign vector as a +-1.0 table, shared by every row of this CTA
+    for (int i = threadIdx.x; i < G::N; i += blockDim.x) sgn[i] = a.pre_signs[i] < 0 ? -1.0f : 1.0f;
+  }
   if (threadIdx.x == 0) {
     for (int s = 0; s < C::S; ++s) {
       mbar_init(&full[s], 1);
@@ -122,9 +128,11 @@ __global__ void __launch_bounds__(StreamCfg<LOGN, Tin>::THREADS, 1) k_rows_strea
         bf16x2_to_f32(v.x, x[4 * j], x[4 * j + 1]);
         bf16x2_to_f32(v.y, x[4 * j + 2], x[4 * j + 3]);
       }
-      if (a.pre_signs != nullptr)
-        apply_sign4(x[4 * j], x[4 * j + 1], x[4 * j + 2], x[4 * j + 3],
-                    __ldg(reinterpret_cast<const uint32_t*>(a.pre_signs + i0)));
+      if (has_signs) {
+        const float4 sv = reinterpret_cast<const float4*>(sgn)[i0 >> 2];
+        mul_x2(x[4 * j], x[4 * j + 1], sv.x, sv.y);
+        mul_x2(x[4 * j + 2], x[4 * j + 3], sv.z, sv.w);
+      }
     }
     reg_stages<G::E, 0, G::LOGE>(x);
     stream_team_sync<LOGN, Tin>(team);  // every thread has read its layout-A data
