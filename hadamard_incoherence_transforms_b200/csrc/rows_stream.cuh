@@ -19,17 +19,20 @@ namespace hit {
 
 __device__ unsigned int g_wait_timeouts = 0;
 
-// Consumer warps per CTA (plus one producer warp).  Eight warps in total keep
-// at most two warps per SM sub-partition, which leaves each thread the full
-// 255 registers for its 128 row elements.
+// Warps per CTA: one producer plus consumers.  Seven warps keep at most two
+// warps per SM sub-partition, which leaves each thread the full 255 registers
+// for its row elements.
 #ifndef HIT_STREAM_WARPS
-#define HIT_STREAM_WARPS 8
-#endif
-// Bytes of shared memory given to the ring of row slots.
-#ifndef HIT_STREAM_RING_BYTES
-#define HIT_STREAM_RING_BYTES (200 * 1024)
+#define HIT_STREAM_WARPS 7
 #endif
 
+// Ring protocol.  Row k of this CTA goes to slot k % S and is consumed by team
+// k % TEAMS.  S is a multiple of TEAMS, so every slot is always served by the
+// same team, which takes the slot's phases strictly in order: when a team
+// waits for phase j of a slot's "full" barrier it has itself consumed phase
+// j-1, and the producer refills a slot only after its "empty" barrier
+// completed the previous phase.  A parity wait therefore never sees a barrier
+// two phases behind or ahead of the phase it asks for.
 template <int LOGN, typename Tin>
 struct StreamCfg {
   using G = Geom<LOGN>;
@@ -40,10 +43,12 @@ struct StreamCfg {
   static constexpr uint32_t SLOT = uint32_t(G::N) * 4;         // fp32 row (transpose space)
   static constexpr uint32_t ROW = uint32_t(G::N) * sizeof(Tin);
   static constexpr uint32_t SIGNS = uint32_t(G::N) * 4;        // +-1.0 per column
-  static constexpr int S = (HIT_STREAM_RING_BYTES - SIGNS) / SLOT;  // ring depth
+  static constexpr uint32_t SMEM_MAX = 232448;                 // opt-in limit per CTA on sm_100
+  static constexpr int S = TEAMS * int((SMEM_MAX - 1024 - SIGNS) / (SLOT * TEAMS));  // ring depth
   static constexpr size_t SMEM = 1024 + SIGNS + size_t(S) * SLOT;
   static constexpr int THREADS = (NCW + 1) * 32;
-  static_assert(S >= 2, "ring needs at least two slots");
+  static_assert(TEAMS >= 1 && S >= TEAMS && S % TEAMS == 0, "ring depth must be a multiple of the team count");
+  static_assert(2 * S * 8 <= 1024, "barriers must fit in the first kilobyte");
 };
 
 template <int LOGN, typename Tin>
