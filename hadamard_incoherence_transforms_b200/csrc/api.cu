@@ -78,6 +78,21 @@ bool use_stream(int logn, const void* x, int64_t ld, int dt) {
 int run_cols(const void* src, int dt_src, int64_t ld_src, void* dst, int dt_dst, int64_t ld_dst, int64_t m,
              int64_t cols, const int8_t* pre, const int8_t* post, float* tmp, int64_t ld_tmp, cudaStream_t st) {
   const int k = ilog2(m);
+  // One pass over whole 4-column strips when the strip rows are vector aligned.
+  if (k >= 8 && k <= 13 && cols % 4 == 0 && ld_src % 4 == 0 && ld_dst % 4 == 0 &&
+      aligned(src, 4 * esize(dt_src)) && aligned(dst, 4 * esize(dt_dst))) {
+    hit::ColArgs a;
+    a.x = src;
+    a.y = dst;
+    a.m = m;
+    a.cols = cols;
+    a.ldx = ld_src;
+    a.ldy = ld_dst;
+    a.pre_signs = pre;
+    a.post_signs = post;
+    a.norm = inv_sqrt(m);
+    return cuda_status(hit::launch_cols_full(k, dt_src, dt_dst, a, st), "column transform launch");
+  }
   const int np = k == 0 ? 1 : (k + 6) / 7;
   int lo = 0;
   for (int p = 0; p < np; ++p) {

@@ -11,9 +11,11 @@
 // last applies 1/sqrt(m) and, for the inverse, the signs before the store.
 // Each thread reads all its elements before writing them and the threads'
 // element sets are disjoint, so a pass may run in place.
+#include <atomic>
+
 #include "device.cuh"
 #include "internal.h"
-#include "rows.cuh"
+#include "rows_ops.cuh"
 
 namespace hit {
 
@@ -48,6 +50,175 @@ __global__ void __launch_bounds__(128) k_cols_pass(const ColArgs a) {
     if (a.post_signs != nullptr && a.post_signs[r] < 0) f = -f;
     dst[r * a.ldy + col] = from_f32<Tout>(f);
   }
+}
+
+// ---------------------------------------------------------------------------
+// Single-pass column transform for 2^8 <= m <= 2^13.
+//
+// A CTA owns complete columns: a strip of 4 adjacent columns per team of
+// T = m/32 threads (256 / T strips per CTA, 256 threads).  Every element moves
+// as part of a 4-column vector (one 16-byte fp32 / 8-byte bf16 access per
+// row), and a thread holds 32 rows x 4 columns = 128 values.  The row index
+// bits are processed in windows of five bits from the top: in phase p the
+// thread's 32 rows differ in the window's bits (register bits), while its
+// thread index supplies the other bits.  Between phases the strip goes
+// through shared memory (row r of a strip is 16-byte chunk r, stored at
+// r ^ ((r >> 5) & 7)).  The last window is widened down to bit 0 and only runs
+// the stages not done yet.  The strip's data crosses HBM exactly once in each
+// direction.
+// ---------------------------------------------------------------------------
+template <int LOGM>
+struct ColFull {
+  static constexpr int M = 1 << LOGM;
+  static constexpr int LOGT = LOGM - 5;
+  static constexpr int T = 1 << LOGT;   // threads per strip
+  static constexpr int STRIPS = 256 / T; // strips per CTA
+  static constexpr int NP = (LOGM + 4) / 5;
+  static constexpr size_t SMEM = size_t(256) * 32 * 16;  // 128 KB
+};
+
+// window (lowest register bit) of phase P
+template <int LOGM, int P>
+struct ColWin {
+  static constexpr int HI = LOGM - 5 * P;                  // exclusive top of the window
+  static constexpr int LO = HI - 5 > 0 ? HI - 5 : 0;       // register window [LO, LO+5)
+  static constexpr int STAGE_LO = HI - 5 > 0 ? 0 : LO;     // new stages: window bits below HI
+  static constexpr int NSTAGE = HI - LO;                   // bits of the window still to do
+};
+
+template <int LOGM, int P>
+__device__ __forceinline__ int64_t colfull_row(int t, int k) {
+  constexpr int LO = ColWin<LOGM, P>::LO;
+  const int low = t & ((1 << LO) - 1);
+  const int high = t >> LO;
+  return int64_t(low | (k << LO) | (high << (LO + 5)));
+}
+
+__device__ __forceinline__ int colfull_chunk(int r) { return r ^ ((r >> 5) & 7); }
+
+template <int LOGM, int P>
+__device__ __forceinline__ void colfull_stages(float (&x)[128]) {
+  // register index 4k + c; row-window bit q <-> register bit q + 2
+  reg_stages<128, 2, 2 + ColWin<LOGM, P>::NSTAGE>(x);
+}
+
+template <int LOGM, int P>
+__device__ __forceinline__ void colfull_get(const float4* strip, float (&x)[128], int t) {
+#pragma unroll
+  for (int k = 0; k < 32; ++k) {
+    const float4 v = strip[colfull_chunk(int(colfull_row<LOGM, P>(t, k)))];
+    x[4 * k] = v.x;
+    x[4 * k + 1] = v.y;
+    x[4 * k + 2] = v.z;
+    x[4 * k + 3] = v.w;
+  }
+}
+template <int LOGM, int P>
+__device__ __forceinline__ void colfull_put(float4* strip, const float (&x)[128], int t) {
+#pragma unroll
+  for (int k = 0; k < 32; ++k)
+    strip[colfull_chunk(int(colfull_row<LOGM, P>(t, k)))] = make_float4(x[4 * k], x[4 * k + 1], x[4 * k + 2], x[4 * k + 3]);
+}
+
+template <int LOGM, typename Tin, typename Tout>
+__global__ void __launch_bounds__(256, 1) k_cols_full(const ColArgs a) {
+  using F = ColFull<LOGM>;
+  extern __shared__ float4 cf_smem[];
+  const int tid = threadIdx.x;
+  const int strip_in_cta = tid >> F::LOGT;
+  const int t = tid & (F::T - 1);
+  const int64_t col0 = (int64_t(blockIdx.x) * F::STRIPS + strip_in_cta) * 4;
+  const bool active = col0 < a.cols;
+  float4* strip = cf_smem + size_t(strip_in_cta) * F::M;
+  float x[128];
+  if (active) {
+    const Tin* src = static_cast<const Tin*>(a.x) + col0;
+#pragma unroll
+    for (int k = 0; k < 32; ++k) {
+      const int64_t r = colfull_row<LOGM, 0>(t, k);
+      float v0, v1, v2, v3;
+      if constexpr (std::is_same<Tin, float>::value) {
+        const float4 v = __ldcs(reinterpret_cast<const float4*>(src + r * a.ldx));
+        v0 = v.x; v1 = v.y; v2 = v.z; v3 = v.w;
+      } else {
+        const uint2 v = __ldcs(reinterpret_cast<const uint2*>(src + r * a.ldx));
+        bf16x2_to_f32(v.x, v0, v1);
+        bf16x2_to_f32(v.y, v2, v3);
+      }
+      if (a.pre_signs != nullptr && a.pre_signs[r] < 0) {
+        v0 = -v0; v1 = -v1; v2 = -v2; v3 = -v3;
+      }
+      x[4 * k] = v0; x[4 * k + 1] = v1; x[4 * k + 2] = v2; x[4 * k + 3] = v3;
+    }
+    colfull_stages<LOGM, 0>(x);
+  }
+  if constexpr (F::NP > 1) {
+    if (active) colfull_put<LOGM, 0>(strip, x, t);
+    __syncthreads();
+    if (active) {
+      colfull_get<LOGM, 1>(strip, x, t);
+      colfull_stages<LOGM, 1>(x);
+    }
+  }
+  if constexpr (F::NP > 2) {
+    __syncthreads();  // all phase-1 reads done before the phase-1 writes
+    if (active) colfull_put<LOGM, 1>(strip, x, t);
+    __syncthreads();
+    if (active) {
+      colfull_get<LOGM, 2>(strip, x, t);
+      colfull_stages<LOGM, 2>(x);
+    }
+  }
+  if (!active) return;
+  constexpr int PL = F::NP - 1;
+  Tout* dst = static_cast<Tout*>(a.y) + col0;
+#pragma unroll
+  for (int k = 0; k < 32; ++k) {
+    const int64_t r = colfull_row<LOGM, PL>(t, k);
+    float v0 = x[4 * k] * a.norm, v1 = x[4 * k + 1] * a.norm, v2 = x[4 * k + 2] * a.norm, v3 = x[4 * k + 3] * a.norm;
+    if (a.post_signs != nullptr && a.post_signs[r] < 0) {
+      v0 = -v0; v1 = -v1; v2 = -v2; v3 = -v3;
+    }
+    if constexpr (std::is_same<Tout, float>::value) {
+      __stcs(reinterpret_cast<float4*>(dst + r * a.ldy), make_float4(v0, v1, v2, v3));
+    } else {
+      __stcs(reinterpret_cast<uint2*>(dst + r * a.ldy), make_uint2(f32_to_bf16x2(v0, v1), f32_to_bf16x2(v2, v3)));
+    }
+  }
+}
+
+template <int LOGM, typename Tin, typename Tout>
+static cudaError_t launch_full_t(const ColArgs& a, cudaStream_t st) {
+  using F = ColFull<LOGM>;
+  auto kern = k_cols_full<LOGM, Tin, Tout>;
+  static std::atomic<unsigned long long> done{0};
+  cudaError_t e = set_smem_attr(kern, F::SMEM, done);
+  if (e != cudaSuccess) return e;
+  const int64_t strips = (a.cols + 3) / 4;
+  const int64_t grid = (strips + F::STRIPS - 1) / F::STRIPS;
+  if (grid > 0x7fffffffLL) return cudaErrorInvalidConfiguration;
+  kern<<<dim3(unsigned(grid)), 256, F::SMEM, st>>>(a);
+  return cudaGetLastError();
+}
+
+template <int LOGM>
+static cudaError_t launch_full_m(int dt_in, int dt_out, const ColArgs& a, cudaStream_t st) {
+  if (dt_in == DT_F32 && dt_out == DT_F32) return launch_full_t<LOGM, float, float>(a, st);
+  if (dt_in == DT_F32) return launch_full_t<LOGM, float, __nv_bfloat16>(a, st);
+  if (dt_out == DT_F32) return launch_full_t<LOGM, __nv_bfloat16, float>(a, st);
+  return launch_full_t<LOGM, __nv_bfloat16, __nv_bfloat16>(a, st);
+}
+
+cudaError_t launch_cols_full(int logm, int dt_in, int dt_out, const ColArgs& a, cudaStream_t st) {
+  switch (logm) {
+    case 8: return launch_full_m<8>(dt_in, dt_out, a, st);
+    case 9: return launch_full_m<9>(dt_in, dt_out, a, st);
+    case 10: return launch_full_m<10>(dt_in, dt_out, a, st);
+    case 11: return launch_full_m<11>(dt_in, dt_out, a, st);
+    case 12: return launch_full_m<12>(dt_in, dt_out, a, st);
+    case 13: return launch_full_m<13>(dt_in, dt_out, a, st);
+  }
+  return cudaErrorInvalidValue;
 }
 
 template <int NB>

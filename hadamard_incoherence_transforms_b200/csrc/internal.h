@@ -55,6 +55,9 @@ struct ColArgs {
   float norm = 1.0f;  // applied on store when != 1
 };
 cudaError_t launch_cols_pass(int nb, int dt_in, int dt_out, const ColArgs& a, cudaStream_t st);
+// Whole column transform in one pass for 2^8 <= m <= 2^13 (4-column strips;
+// needs cols % 4 == 0 and 16-byte (fp32) / 8-byte (bf16) aligned strip rows).
+cudaError_t launch_cols_full(int logm, int dt_in, int dt_out, const ColArgs& a, cudaStream_t st);
 
 // One mixed-radix butterfly stage (see butterfly_apply in hit.h).
 struct StageArgs {

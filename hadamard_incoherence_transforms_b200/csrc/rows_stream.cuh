@@ -42,7 +42,7 @@ struct StreamCfg {
   static constexpr int TEAMS = NCW / WPR;                      // rows in compute at once
   static constexpr uint32_t SLOT = uint32_t(G::N) * 4;         // fp32 row (transpose space)
   static constexpr uint32_t ROW = uint32_t(G::N) * sizeof(Tin);
-  static constexpr uint32_t SIGNS = uint32_t(G::N) * 4;        // +-1.0 per column
+  static constexpr uint32_t SIGNS = uint32_t(G::N) * 4;        // sign-bit mask per column
   static constexpr uint32_t SMEM_MAX = 232448;                 // opt-in limit per CTA on sm_100
   static constexpr int S = TEAMS * int((SMEM_MAX - 1024 - SIGNS) / (SLOT * TEAMS));  // ring depth
   static constexpr size_t SMEM = 1024 + SIGNS + size_t(S) * SLOT;
@@ -67,12 +67,12 @@ __global__ void __launch_bounds__(StreamCfg<LOGN, Tin>::THREADS, 1) k_rows_strea
   extern __shared__ __align__(1024) uint8_t smem[];
   uint64_t* full = reinterpret_cast<uint64_t*>(smem);
   uint64_t* empty = full + C::S;
-  float* sgn = reinterpret_cast<float*>(smem + 1024);
+  uint32_t* sgn = reinterpret_cast<uint32_t*>(smem + 1024);
   uint8_t* slots = smem + 1024 + C::SIGNS;
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const bool has_signs = a.pre_signs != nullptr;
-  if (has_signs) {  // the sign vector as a +-1.0 table, shared by every row of this CTA
-    for (int i = threadIdx.x; i < G::N; i += blockDim.x) sgn[i] = a.pre_signs[i] < 0 ? -1.0f : 1.0f;
+  if (has_signs) {  // the sign vector as sign-bit masks, shared by every row of this CTA
+    for (int i = threadIdx.x; i < G::N; i += blockDim.x) sgn[i] = a.pre_signs[i] < 0 ? 0x80000000u : 0u;
   }
   if (threadIdx.x == 0) {
     for (int s = 0; s < C::S; ++s) {
@@ -133,10 +133,12 @@ __global__ void __launch_bounds__(StreamCfg<LOGN, Tin>::THREADS, 1) k_rows_strea
         bf16x2_to_f32(v.x, x[4 * j], x[4 * j + 1]);
         bf16x2_to_f32(v.y, x[4 * j + 2], x[4 * j + 3]);
       }
-      if (has_signs) {
-        const float4 sv = reinterpret_cast<const float4*>(sgn)[i0 >> 2];
-        mul_x2(x[4 * j], x[4 * j + 1], sv.x, sv.y);
-        mul_x2(x[4 * j + 2], x[4 * j + 3], sv.z, sv.w);
+      if (has_signs) {  // xor of the sign bit runs on the integer pipe, not the FP32 pipe
+        const uint4 sv = reinterpret_cast<const uint4*>(sgn)[i0 >> 2];
+        x[4 * j] = __uint_as_float(__float_as_uint(x[4 * j]) ^ sv.x);
+        x[4 * j + 1] = __uint_as_float(__float_as_uint(x[4 * j + 1]) ^ sv.y);
+        x[4 * j + 2] = __uint_as_float(__float_as_uint(x[4 * j + 2]) ^ sv.z);
+        x[4 * j + 3] = __uint_as_float(__float_as_uint(x[4 * j + 3]) ^ sv.w);
       }
     }
     reg_stages<G::E, 0, G::LOGE>(x);
