@@ -5,6 +5,7 @@
 #include <cstdarg>
 #include <cstdio>
 #include <string>
+#include <vector>
 
 #include "hit.h"
 #include "internal.h"
@@ -174,6 +175,79 @@ int rht_impl(bool inverse, const void* x, void* y, int64_t rows, int64_t n, int6
 
 }  // namespace
 
+// Plan one butterfly pass applying stages order[0..cnt) (consecutive digits).
+static bool plan_pass(const int* order, int cnt, const int32_t* radices, const int64_t* S, const float* const* blocks,
+                      const int64_t* n_groups, int64_t len, int64_t outer, int axis, bool transpose,
+                      hit::BflyPass& p) {
+  if (cnt > hit::kMaxPassStages) return false;
+  int dlo = order[0], dhi = order[0];
+  for (int k = 1; k < cnt; ++k) {
+    dlo = order[k] < dlo ? order[k] : dlo;
+    dhi = order[k] > dhi ? order[k] : dhi;
+  }
+  int64_t P = 1;
+  for (int t = dlo; t <= dhi; ++t) P *= radices[t];
+  if (P > 16384) return false;
+  const int64_t S_in = S[dhi];
+  const size_t budget = 200 * 1024;
+  // consecutive lo values per tile: along rows they are contiguous in memory
+  int NL = 1;
+  if (axis == 1)
+    for (int c = 8; c >= 1; --c)
+      if (S_in % c == 0) {
+        NL = c;
+        break;
+      }
+  for (; NL >= 1; NL = (NL > 1 ? NL / 2 : 0)) {
+    if (S_in % NL) continue;
+    int64_t blk = 0;
+    for (int k = 0; k < cnt; ++k) {
+      const int t = order[k];
+      const int64_t b = radices[t];
+      const bool shared = n_groups[t] == 1 && len / b != 1;
+      blk += shared ? b * b : P * NL * b;
+    }
+    const int64_t pnl = P * NL;
+    const int64_t pitch = (pnl % 2 == 0) ? pnl + 1 : pnl;
+    const int nb_try[] = {32, 16, 8, 4, 2, 1};
+    for (int nb : nb_try) {
+      const size_t bytes = static_cast<size_t>(blk + nb * pitch) * sizeof(float);
+      if (bytes > budget) continue;
+      p = hit::BflyPass();
+      p.outer = outer;
+      p.axis = axis;
+      p.P = static_cast<int>(P);
+      p.S_in = S_in;
+      p.NL = NL;
+      p.NB = nb;
+      p.pitch = static_cast<int>(pitch);
+      p.n_tiles = (len / (P * S_in)) * (S_in / NL);
+      p.blk_floats = static_cast<int>(blk);
+      p.ns = cnt;
+      int ofs = 0;
+      for (int k = 0; k < cnt; ++k) {
+        const int t = order[k];
+        hit::BflyStage& st = p.st[k];
+        st.blocks = blocks[t];
+        st.b = radices[t];
+        st.ls = static_cast<int>(S[t] / S_in);
+        st.sofs = ofs;
+        st.shared_block = (n_groups[t] == 1 && len / radices[t] != 1) ? 1 : 0;
+        st.transpose = transpose ? 1 : 0;
+        ofs += st.shared_block ? st.b * st.b : static_cast<int>(P * NL * st.b);
+      }
+      // enough CTAs to fill the machine a few times over
+      const int64_t chunks = (outer + nb - 1) / nb;
+      int64_t splits = (4 * 148 + p.n_tiles - 1) / p.n_tiles;
+      splits = splits < 1 ? 1 : (splits > chunks ? chunks : splits);
+      p.chunks_per_split = (chunks + splits - 1) / splits;
+      return true;
+    }
+    if (NL == 1) break;
+  }
+  return false;
+}
+
 extern "C" {
 
 int hit_version(void) { return 100; }
@@ -263,25 +337,50 @@ int butterfly_apply(const void* x, void* y, int64_t rows, int64_t n, int64_t ldx
       ld_tmp = n;
     }
   }
-  for (int p = 0; p < n_stages; ++p) {
-    const int t = transpose ? n_stages - 1 - p : p;
-    int64_t stride = 1;
-    for (int u = t + 1; u < n_stages; ++u) stride *= radices[u];
-    hit::StageArgs a;
-    const bool first = p == 0, last = p == n_stages - 1;
-    a.x = first ? x : tmp;
-    a.ldx = first ? ldx : ld_tmp;
-    a.y = last ? y : tmp;
-    a.ldy = last ? ldy : ld_tmp;
-    a.outer = axis == 1 ? rows : n;
-    a.len = len;
-    a.axis = axis;
-    a.b = radices[t];
-    a.stride = stride;
-    a.blocks = blocks[t];
-    a.shared_block = n_groups[t] == 1 && len / radices[t] != 1 ? 1 : 0;
-    a.transpose = transpose ? 1 : 0;
-    const cudaError_t e = hit::launch_butterfly_stage(first ? dtype_in : HIT_F32, last ? dtype_out : HIT_F32, a, st);
+  // Strides, then group consecutive stages (in application order) into passes
+  // whose tile and blocks fit the shared-memory budget.
+  int64_t S[16];
+  {
+    int64_t acc = 1;
+    for (int t = n_stages - 1; t >= 0; --t) {
+      S[t] = acc;
+      acc *= radices[t];
+    }
+  }
+  int order[16];
+  for (int i = 0; i < n_stages; ++i) order[i] = transpose ? n_stages - 1 - i : i;
+  const int64_t outer = axis == 1 ? rows : n;
+  std::vector<hit::BflyPass> passes;
+  int i = 0;
+  while (i < n_stages) {
+    hit::BflyPass best;
+    bool have = false;
+    for (int j = i; j < n_stages; ++j) {  // try to extend the run [i, j]
+      hit::BflyPass cand;
+      if (!plan_pass(order + i, j - i + 1, radices, S, blocks, n_groups, len, outer, axis, transpose != 0, cand))
+        break;
+      best = cand;
+      have = true;
+    }
+    if (!have) return fail(HIT_EUNSUPPORTED, "%s: stage %d does not fit in shared memory", fn, order[i]);
+    passes.push_back(best);
+    i += best.ns;
+  }
+  const int np = static_cast<int>(passes.size());
+  for (int q = 0; q < np; ++q) {
+    hit::BflyPass& p = passes[q];
+    const bool first = q == 0, last = q == np - 1;
+    p.x = first ? x : tmp;
+    p.ldx = first ? ldx : ld_tmp;
+    p.y = last ? y : tmp;
+    p.ldy = last ? ldy : ld_tmp;
+    if (!first || !last) {
+      if (tmp == nullptr) {  // several passes but a single stage run was expected
+        const size_t need = static_cast<size_t>(rows) * static_cast<size_t>(n) * 4;
+        return fail(HIT_EWORKSPACE, "%s: needs %zu workspace bytes", fn, need);
+      }
+    }
+    const cudaError_t e = hit::launch_butterfly_pass(first ? dtype_in : HIT_F32, last ? dtype_out : HIT_F32, p, st);
     if (e != cudaSuccess) return cuda_status(e, fn);
   }
   return HIT_OK;

@@ -59,20 +59,34 @@ cudaError_t launch_cols_pass(int nb, int dt_in, int dt_out, const ColArgs& a, cu
 // needs cols % 4 == 0 and 16-byte (fp32) / 8-byte (bf16) aligned strip rows).
 cudaError_t launch_cols_full(int logm, int dt_in, int dt_out, const ColArgs& a, cudaStream_t st);
 
-// One mixed-radix butterfly stage (see butterfly_apply in hit.h).
-struct StageArgs {
+// One pass of mixed-radix butterfly stages over consecutive digits (see
+// butterfly.cu for the tiling).
+struct BflyStage {
+  const float* blocks = nullptr;  // [G, b, b] fp32, or one shared block
+  int b = 1;                      // radix
+  int ls = 1;                     // stride of this digit inside the group index mid
+  int sofs = 0;                   // float offset of the stage's blocks in shared memory
+  int shared_block = 0;
+  int transpose = 0;              // use B^T
+};
+constexpr int kMaxPassStages = 16;
+struct BflyPass {
   const void* x = nullptr;
   void* y = nullptr;
-  int64_t outer = 0;        // rows (axis 1) or columns (axis 0)
-  int64_t len = 0;          // transform length
+  int64_t outer = 0;          // rows (axis 1) or columns (axis 0)
   int64_t ldx = 0, ldy = 0;
   int axis = 1;
-  int b = 1;                // radix of this stage
-  int64_t stride = 1;       // S_t = product of the later radices
-  const float* blocks = nullptr;  // [G, b, b]
-  int shared_block = 0;     // 1: one block for all groups
-  int transpose = 0;        // use B^T
+  int P = 1;                  // positions per group (product of the pass's radices)
+  int64_t S_in = 1;           // stride of the pass's last digit
+  int NL = 1;                 // consecutive lo values per tile
+  int NB = 1;                 // rows / columns per chunk
+  int pitch = 1;              // floats per tile row in shared memory (odd)
+  int64_t n_tiles = 1;
+  int64_t chunks_per_split = 1;
+  int blk_floats = 0;
+  int ns = 0;
+  BflyStage st[kMaxPassStages];
 };
-cudaError_t launch_butterfly_stage(int dt_in, int dt_out, const StageArgs& a, cudaStream_t st);
+cudaError_t launch_butterfly_pass(int dt_in, int dt_out, const BflyPass& p, cudaStream_t st);
 
 }  // namespace hit
