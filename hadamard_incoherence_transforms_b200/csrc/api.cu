@@ -79,9 +79,24 @@ bool use_stream(int logn, const void* x, int64_t ld, int dt) {
 int run_cols(const void* src, int dt_src, int64_t ld_src, void* dst, int dt_dst, int64_t ld_dst, int64_t m,
              int64_t cols, const int8_t* pre, const int8_t* post, float* tmp, int64_t ld_tmp, cudaStream_t st) {
   const int k = ilog2(m);
+  const bool vec_ok = ld_src % 4 == 0 && ld_dst % 4 == 0 && aligned(src, 4 * esize(dt_src)) &&
+                      aligned(dst, 4 * esize(dt_dst));
+  // One pass with clusters over 32-column strips.
+  if (k >= 10 && k <= 13 && cols % 32 == 0 && vec_ok) {
+    hit::ColArgs a;
+    a.x = src;
+    a.y = dst;
+    a.m = m;
+    a.cols = cols;
+    a.ldx = ld_src;
+    a.ldy = ld_dst;
+    a.pre_signs = pre;
+    a.post_signs = post;
+    a.norm = inv_sqrt(m);
+    return cuda_status(hit::launch_cols_cluster(k, dt_src, dt_dst, a, st), "column transform launch");
+  }
   // One pass over whole 4-column strips when the strip rows are vector aligned.
-  if (k >= 8 && k <= 13 && cols % 4 == 0 && ld_src % 4 == 0 && ld_dst % 4 == 0 &&
-      aligned(src, 4 * esize(dt_src)) && aligned(dst, 4 * esize(dt_dst))) {
+  if (k >= 8 && k <= 13 && cols % 4 == 0 && vec_ok) {
     hit::ColArgs a;
     a.x = src;
     a.y = dst;
@@ -190,27 +205,24 @@ static bool plan_pass(const int* order, int cnt, const int32_t* radices, const i
   if (P > 16384) return false;
   const int64_t S_in = S[dhi];
   const size_t budget = 200 * 1024;
-  // consecutive lo values per tile: along rows they are contiguous in memory
-  int NL = 1;
+  // consecutive lo values per tile (a power of two dividing S_in); along rows
+  // they are contiguous in memory, so up to eight of them per tile
+  int log_nl = 0;
   if (axis == 1)
-    for (int c = 8; c >= 1; --c)
-      if (S_in % c == 0) {
-        NL = c;
-        break;
-      }
-  for (; NL >= 1; NL = (NL > 1 ? NL / 2 : 0)) {
-    if (S_in % NL) continue;
+    while (log_nl < 3 && S_in % (int64_t(2) << log_nl) == 0) ++log_nl;
+  for (; log_nl >= 0; --log_nl) {
+    const int NL = 1 << log_nl;
     int64_t blk = 0;
     for (int k = 0; k < cnt; ++k) {
       const int t = order[k];
-      const int64_t b = radices[t];
+      const int64_t b = radices[t], bp = (b + 3) / 4 * 4;
       const bool shared = n_groups[t] == 1 && len / b != 1;
-      blk += shared ? b * b : P * NL * b;
+      blk += (shared ? 1 : (P / b) * NL) * b * bp;
     }
     const int64_t pnl = P * NL;
     const int64_t pitch = (pnl % 2 == 0) ? pnl + 1 : pnl;
-    const int nb_try[] = {32, 16, 8, 4, 2, 1};
-    for (int nb : nb_try) {
+    for (int log_nb = 5; log_nb >= 0; --log_nb) {
+      const int nb = 1 << log_nb;
       const size_t bytes = static_cast<size_t>(blk + nb * pitch) * sizeof(float);
       if (bytes > budget) continue;
       p = hit::BflyPass();
@@ -219,7 +231,10 @@ static bool plan_pass(const int* order, int cnt, const int32_t* radices, const i
       p.P = static_cast<int>(P);
       p.S_in = S_in;
       p.NL = NL;
+      p.log_nl = log_nl;
       p.NB = nb;
+      p.log_nb = log_nb;
+      p.div_pnl = hit::make_fastdiv(static_cast<uint32_t>(pnl));
       p.pitch = static_cast<int>(pitch);
       p.n_tiles = (len / (P * S_in)) * (S_in / NL);
       p.blk_floats = static_cast<int>(blk);
@@ -230,11 +245,13 @@ static bool plan_pass(const int* order, int cnt, const int32_t* radices, const i
         hit::BflyStage& st = p.st[k];
         st.blocks = blocks[t];
         st.b = radices[t];
+        st.bp = (st.b + 3) / 4 * 4;
         st.ls = static_cast<int>(S[t] / S_in);
+        st.div_ls = hit::make_fastdiv(static_cast<uint32_t>(st.ls));
         st.sofs = ofs;
         st.shared_block = (n_groups[t] == 1 && len / radices[t] != 1) ? 1 : 0;
         st.transpose = transpose ? 1 : 0;
-        ofs += st.shared_block ? st.b * st.b : static_cast<int>(P * NL * st.b);
+        ofs += (st.shared_block ? 1 : static_cast<int>((P / st.b) * NL)) * st.b * st.bp;
       }
       // enough CTAs to fill the machine a few times over
       const int64_t chunks = (outer + nb - 1) / nb;
@@ -243,7 +260,6 @@ static bool plan_pass(const int* order, int cnt, const int32_t* radices, const i
       p.chunks_per_split = (chunks + splits - 1) / splits;
       return true;
     }
-    if (NL == 1) break;
   }
   return false;
 }

@@ -11,6 +11,8 @@
 // last applies 1/sqrt(m) and, for the inverse, the signs before the store.
 // Each thread reads all its elements before writing them and the threads'
 // element sets are disjoint, so a pass may run in place.
+#include <cooperative_groups.h>
+
 #include <atomic>
 
 #include "device.cuh"
@@ -217,6 +219,143 @@ cudaError_t launch_cols_full(int logm, int dt_in, int dt_out, const ColArgs& a, 
     case 11: return launch_full_m<11>(dt_in, dt_out, a, st);
     case 12: return launch_full_m<12>(dt_in, dt_out, a, st);
     case 13: return launch_full_m<13>(dt_in, dt_out, a, st);
+  }
+  return cudaErrorInvalidValue;
+}
+
+// ---------------------------------------------------------------------------
+// Column transform for 1024 <= m <= 8192 with thread-block clusters.
+//
+// A cluster of CL = m / 1024 CTAs owns a strip of 32 adjacent columns over
+// all m rows; CTA c of the cluster holds rows [1024 c, 1024 c + 1024) of the
+// strip (128 KB fp32).  Row segments are 32 columns wide (64 B bf16 / 128 B
+// fp32), so global accesses are whole sectors.  Within a CTA a thread owns
+// one 4-column quad and 32 rows: first rows tr + 32k (the register bits are
+// row bits 5..9), then, after one pass through shared memory, rows
+// 32 tr + r (row bits 0..4).  The CL row blocks (row bits 10 and up) are then
+// combined through distributed shared memory: each thread reads the CL
+// vectors of one (row, quad) position from the cluster's CTAs, runs the
+// remaining log2(CL) stages and writes the CL output rows.
+// ---------------------------------------------------------------------------
+template <int CL, typename Tin, typename Tout>
+__global__ void __launch_bounds__(256, 1) k_cols_cluster(const ColArgs a) {
+  extern __shared__ float4 cs_smem[];  // [1024 rows][8 quads]
+  namespace cg = cooperative_groups;
+  cg::cluster_group cluster = cg::this_cluster();
+  const int crank = static_cast<int>(cluster.block_rank());
+  const int64_t col0 = (int64_t(blockIdx.x) / CL) * 32;
+  const int tid = threadIdx.x;
+  const int q = tid & 7;    // column quad within the strip
+  const int tr = tid >> 3;  // 0..31
+  const int64_t row_base = int64_t(crank) * 1024;
+  float x[128];
+  // phase 1: rows tr + 32 k of this CTA's block
+  const Tin* src = static_cast<const Tin*>(a.x) + col0 + 4 * q;
+#pragma unroll
+  for (int k = 0; k < 32; ++k) {
+    const int64_t r = row_base + tr + 32 * k;
+    float v0, v1, v2, v3;
+    if constexpr (std::is_same<Tin, float>::value) {
+      const float4 v = __ldcs(reinterpret_cast<const float4*>(src + r * a.ldx));
+      v0 = v.x; v1 = v.y; v2 = v.z; v3 = v.w;
+    } else {
+      const uint2 v = __ldcs(reinterpret_cast<const uint2*>(src + r * a.ldx));
+      bf16x2_to_f32(v.x, v0, v1);
+      bf16x2_to_f32(v.y, v2, v3);
+    }
+    if (a.pre_signs != nullptr && a.pre_signs[r] < 0) {
+      v0 = -v0; v1 = -v1; v2 = -v2; v3 = -v3;
+    }
+    x[4 * k] = v0; x[4 * k + 1] = v1; x[4 * k + 2] = v2; x[4 * k + 3] = v3;
+  }
+  reg_stages<128, 2, 7>(x);  // row bits 5..9
+#pragma unroll
+  for (int k = 0; k < 32; ++k)
+    cs_smem[(tr + 32 * k) * 8 + q] = make_float4(x[4 * k], x[4 * k + 1], x[4 * k + 2], x[4 * k + 3]);
+  __syncthreads();
+  // phase 2: rows 32 tr + r
+#pragma unroll
+  for (int r = 0; r < 32; ++r) {
+    const float4 v = cs_smem[(32 * tr + r) * 8 + q];
+    x[4 * r] = v.x; x[4 * r + 1] = v.y; x[4 * r + 2] = v.z; x[4 * r + 3] = v.w;
+  }
+  reg_stages<128, 2, 7>(x);  // row bits 0..4
+  __syncthreads();           // every phase-2 read is done before the writes
+#pragma unroll
+  for (int r = 0; r < 32; ++r)
+    cs_smem[(32 * tr + r) * 8 + q] = make_float4(x[4 * r], x[4 * r + 1], x[4 * r + 2], x[4 * r + 3]);
+  cluster.sync();  // all blocks of the strip are in shared memory
+  // phase 3: this CTA combines rows (c', row_low) for row_low in its share
+  Tout* dst = static_cast<Tout*>(a.y) + col0 + 4 * q;
+  constexpr int SHARE = 1024 / CL;
+#pragma unroll 1
+  for (int u = 0; u < SHARE / 32; ++u) {
+    const int row_low = crank * SHARE + tr + 32 * u;
+    float v[4 * CL];
+#pragma unroll
+    for (int c = 0; c < CL; ++c) {
+      const float4* rem = cluster.map_shared_rank(cs_smem, c);
+      const float4 w = rem[row_low * 8 + q];
+      v[4 * c] = w.x; v[4 * c + 1] = w.y; v[4 * c + 2] = w.z; v[4 * c + 3] = w.w;
+    }
+    if constexpr (CL > 1) reg_stages<4 * CL, 2, 2 + (CL == 2 ? 1 : (CL == 4 ? 2 : 3))>(v);
+#pragma unroll
+    for (int c = 0; c < CL; ++c) {
+      const int64_t r = int64_t(c) * 1024 + row_low;
+      float o0 = v[4 * c] * a.norm, o1 = v[4 * c + 1] * a.norm, o2 = v[4 * c + 2] * a.norm, o3 = v[4 * c + 3] * a.norm;
+      if (a.post_signs != nullptr && a.post_signs[r] < 0) {
+        o0 = -o0; o1 = -o1; o2 = -o2; o3 = -o3;
+      }
+      if constexpr (std::is_same<Tout, float>::value) {
+        __stcs(reinterpret_cast<float4*>(dst + r * a.ldy), make_float4(o0, o1, o2, o3));
+      } else {
+        __stcs(reinterpret_cast<uint2*>(dst + r * a.ldy), make_uint2(f32_to_bf16x2(o0, o1), f32_to_bf16x2(o2, o3)));
+      }
+    }
+  }
+  cluster.sync();  // no CTA leaves while others still read its shared memory
+}
+
+template <int CL, typename Tin, typename Tout>
+static cudaError_t launch_cluster_t(const ColArgs& a, cudaStream_t st) {
+  auto kern = k_cols_cluster<CL, Tin, Tout>;
+  constexpr size_t smem = size_t(1024) * 8 * sizeof(float4);
+  static std::atomic<unsigned long long> done{0};
+  cudaError_t e = set_smem_attr(kern, smem, done);
+  if (e != cudaSuccess) return e;
+  const int64_t strips = a.cols / 32;
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(static_cast<unsigned>(strips * CL));
+  cfg.blockDim = dim3(256);
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = st;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeClusterDimension;
+  attr[0].val.clusterDim.x = CL;
+  attr[0].val.clusterDim.y = 1;
+  attr[0].val.clusterDim.z = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  e = cudaLaunchKernelEx(&cfg, kern, a);
+  if (e != cudaSuccess) return e;
+  return cudaGetLastError();
+}
+
+template <int CL>
+static cudaError_t launch_cluster_cl(int dt_in, int dt_out, const ColArgs& a, cudaStream_t st) {
+  if (dt_in == DT_F32 && dt_out == DT_F32) return launch_cluster_t<CL, float, float>(a, st);
+  if (dt_in == DT_F32) return launch_cluster_t<CL, float, __nv_bfloat16>(a, st);
+  if (dt_out == DT_F32) return launch_cluster_t<CL, __nv_bfloat16, float>(a, st);
+  return launch_cluster_t<CL, __nv_bfloat16, __nv_bfloat16>(a, st);
+}
+
+cudaError_t launch_cols_cluster(int logm, int dt_in, int dt_out, const ColArgs& a, cudaStream_t st) {
+  if (a.cols % 32 != 0 || a.cols / 32 > 0x7fffffffLL / 8) return cudaErrorInvalidValue;
+  switch (logm) {
+    case 10: return launch_cluster_cl<1>(dt_in, dt_out, a, st);
+    case 11: return launch_cluster_cl<2>(dt_in, dt_out, a, st);
+    case 12: return launch_cluster_cl<4>(dt_in, dt_out, a, st);
+    case 13: return launch_cluster_cl<8>(dt_in, dt_out, a, st);
   }
   return cudaErrorInvalidValue;
 }

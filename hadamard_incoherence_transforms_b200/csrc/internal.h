@@ -58,13 +58,33 @@ cudaError_t launch_cols_pass(int nb, int dt_in, int dt_out, const ColArgs& a, cu
 // Whole column transform in one pass for 2^8 <= m <= 2^13 (4-column strips;
 // needs cols % 4 == 0 and 16-byte (fp32) / 8-byte (bf16) aligned strip rows).
 cudaError_t launch_cols_full(int logm, int dt_in, int dt_out, const ColArgs& a, cudaStream_t st);
+// Whole column transform for 2^10 <= m <= 2^13 with thread-block clusters of
+// m/1024 CTAs (32-column strips; needs cols % 32 == 0, aligned strip rows).
+cudaError_t launch_cols_cluster(int logm, int dt_in, int dt_out, const ColArgs& a, cudaStream_t st);
 
 // One pass of mixed-radix butterfly stages over consecutive digits (see
 // butterfly.cu for the tiling).
+// Unsigned division by a run-time constant d (d >= 1, numerators < 2^31):
+// q = (umulhi(n, mul) + n) >> shr.
+struct FastDiv {
+  uint32_t d = 1, mul = 0, shr = 0;
+};
+inline FastDiv make_fastdiv(uint32_t d) {
+  FastDiv f;
+  f.d = d;
+  uint32_t s = 0;
+  while ((1ull << s) < d) ++s;
+  f.shr = s;
+  f.mul = static_cast<uint32_t>(((1ull << 32) * ((1ull << s) - d)) / d + 1);
+  if (d == 1) f.mul = 0;
+  return f;
+}
 struct BflyStage {
   const float* blocks = nullptr;  // [G, b, b] fp32, or one shared block
   int b = 1;                      // radix
+  int bp = 4;                     // b rounded up to a multiple of 4 (shared-memory row length)
   int ls = 1;                     // stride of this digit inside the group index mid
+  FastDiv div_ls;                 // division by ls
   int sofs = 0;                   // float offset of the stage's blocks in shared memory
   int shared_block = 0;
   int transpose = 0;              // use B^T
@@ -78,8 +98,11 @@ struct BflyPass {
   int axis = 1;
   int P = 1;                  // positions per group (product of the pass's radices)
   int64_t S_in = 1;           // stride of the pass's last digit
-  int NL = 1;                 // consecutive lo values per tile
-  int NB = 1;                 // rows / columns per chunk
+  int NL = 1;                 // consecutive lo values per tile (power of two)
+  int log_nl = 0;
+  int NB = 1;                 // rows / columns per chunk (power of two)
+  int log_nb = 0;
+  FastDiv div_pnl;            // division by P * NL
   int pitch = 1;              // floats per tile row in shared memory (odd)
   int64_t n_tiles = 1;
   int64_t chunks_per_split = 1;

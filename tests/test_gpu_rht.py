@@ -108,3 +108,17 @@ def test_activation_workload_full_size():
     # full-row check of a few rows
     rows = np.array([0, 1, 4095, 8191])
     assert_close(host(y[rows.tolist()]), oh.rht_rows(x64[rows], d["signs"]), torch.bfloat16, "rows")
+
+
+@pytest.mark.parametrize("m", [1024, 2048, 4096, 8192])
+@pytest.mark.parametrize("cols", [32, 96])
+@pytest.mark.parametrize("dts", [("f32", "f32"), ("bf16", "f32"), ("f32", "bf16")])
+def test_columns_cluster_path(m, cols, dts):
+    """Column lengths 1024..8192 with 32-column strips (the cluster kernel)."""
+    xin, x64, _ = make_input(m, cols, 4000 + m + cols, DT[dts[0]])
+    s = (np.random.default_rng(m + 1).integers(0, 2, m, dtype=np.int8) * 2 - 1).astype(np.int8)
+    y = hit.rht_forward(xin, to_gpu_i8(s), axis=0, out_dtype=DT[dts[1]])
+    yi = hit.rht_inverse(xin, to_gpu_i8(s), axis=0, out_dtype=DT[dts[1]])
+    torch.cuda.synchronize()
+    assert_close(host(y).T, oh.rht_cols(x64, s).T, DT[dts[1]], f"cluster cols m={m}")
+    assert_close(host(yi).T, oh.irht_cols(x64, s).T, DT[dts[1]], f"cluster inverse cols m={m}")
