@@ -81,8 +81,8 @@ int run_cols(const void* src, int dt_src, int64_t ld_src, void* dst, int dt_dst,
   const int k = ilog2(m);
   const bool vec_ok = ld_src % 4 == 0 && ld_dst % 4 == 0 && aligned(src, 4 * esize(dt_src)) &&
                       aligned(dst, 4 * esize(dt_dst));
-  // One pass with clusters over 32-column strips.
-  if (k >= 10 && k <= 13 && cols % 32 == 0 && vec_ok) {
+  // One pass with clusters over 16-column strips.
+  if (k >= 10 && k <= 13 && cols % 16 == 0 && vec_ok) {
     hit::ColArgs a;
     a.x = src;
     a.y = dst;
@@ -204,7 +204,7 @@ static bool plan_pass(const int* order, int cnt, const int32_t* radices, const i
   for (int t = dlo; t <= dhi; ++t) P *= radices[t];
   if (P > 16384) return false;
   const int64_t S_in = S[dhi];
-  const size_t budget = 200 * 1024;
+  const size_t budget = 100 * 1024;  // two CTAs per SM overlap their load / compute / store phases
   // consecutive lo values per tile (a power of two dividing S_in); along rows
   // they are contiguous in memory, so up to eight of them per tile
   int log_nl = 0;
@@ -221,7 +221,7 @@ static bool plan_pass(const int* order, int cnt, const int32_t* radices, const i
     }
     const int64_t pnl = P * NL;
     const int64_t pitch = (pnl % 2 == 0) ? pnl + 1 : pnl;
-    for (int log_nb = 5; log_nb >= 0; --log_nb) {
+    for (int log_nb = 6; log_nb >= 0; --log_nb) {
       const int nb = 1 << log_nb;
       const size_t bytes = static_cast<size_t>(blk + nb * pitch) * sizeof(float);
       if (bytes > budget) continue;

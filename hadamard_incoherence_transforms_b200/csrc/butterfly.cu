@@ -32,7 +32,7 @@ __device__ __forceinline__ uint32_t fdiv(uint32_t n, const FastDiv& f) {
 }
 
 template <int BM, typename Tin, typename Tout>
-__global__ void __launch_bounds__(256) k_bfly_pass(const BflyPass p) {
+__global__ void __launch_bounds__(256, 2) k_bfly_pass(const BflyPass p) {  // launched with 256 threads, up to two CTAs per SM
   extern __shared__ float4 bf_smem4[];
   float* sblk = reinterpret_cast<float*>(bf_smem4);  // per stage: [group][k][bp] (bp >= b, zero padded)
   float* tile = sblk + p.blk_floats;                  // [NB][pitch]
@@ -78,20 +78,38 @@ __global__ void __launch_bounds__(256) k_bfly_pass(const BflyPass p) {
     if (o0 >= p.outer) break;
     const int nb = int(p.outer - o0 < p.NB ? p.outer - o0 : p.NB);
     __syncthreads();  // blocks ready / previous chunk stored
-    // 2. load the tile (consecutive threads: consecutive memory)
-    for (int e = tid; e < (PNL << p.log_nb); e += blockDim.x) {
-      int bi, q;
-      if (p.axis == 1) {
-        bi = int(fdiv(uint32_t(e), p.div_pnl));
-        q = e - bi * PNL;
-      } else {
-        bi = e & nbm;
-        q = e >> p.log_nb;
+    // 2. load the tile (consecutive threads: consecutive memory),
+    //    sixteen independent loads in flight per thread before they land in shared memory
+    constexpr int U = 16;
+    const int total = PNL << p.log_nb;
+    for (int e0 = tid; e0 < total; e0 += U * blockDim.x) {
+      float val[U];
+      int dst[U];
+#pragma unroll
+      for (int u = 0; u < U; ++u) {
+        const int e = e0 + u * blockDim.x;
+        dst[u] = -1;
+        val[u] = 0.0f;
+        if (e < total) {
+          int bi, q;
+          if (p.axis == 1) {
+            bi = int(fdiv(uint32_t(e), p.div_pnl));
+            q = e - bi * PNL;
+          } else {
+            bi = e & nbm;
+            q = e >> p.log_nb;
+          }
+          if (bi < nb) {
+            const int64_t pos = base + int64_t(q >> p.log_nl) * p.S_in + (q & nlm);
+            const int64_t g = p.axis == 1 ? (o0 + bi) * p.ldx + pos : pos * p.ldx + (o0 + bi);
+            val[u] = to_f32(__ldcs(src + g));
+            dst[u] = bi * p.pitch + q;
+          }
+        }
       }
-      if (bi >= nb) continue;
-      const int64_t pos = base + int64_t(q >> p.log_nl) * p.S_in + (q & nlm);
-      const int64_t g = p.axis == 1 ? (o0 + bi) * p.ldx + pos : pos * p.ldx + (o0 + bi);
-      tile[bi * p.pitch + q] = to_f32(src[g]);
+#pragma unroll
+      for (int u = 0; u < U; ++u)
+        if (dst[u] >= 0) tile[dst[u]] = val[u];
     }
     __syncthreads();
     // 3. the stages, in application order
@@ -134,6 +152,7 @@ __global__ void __launch_bounds__(256) k_bfly_pass(const BflyPass p) {
       __syncthreads();
     }
     // 4. store the tile
+#pragma unroll 4
     for (int e = tid; e < (PNL << p.log_nb); e += blockDim.x) {
       int bi, q;
       if (p.axis == 1) {
@@ -146,7 +165,7 @@ __global__ void __launch_bounds__(256) k_bfly_pass(const BflyPass p) {
       if (bi >= nb) continue;
       const int64_t pos = base + int64_t(q >> p.log_nl) * p.S_in + (q & nlm);
       const int64_t g = p.axis == 1 ? (o0 + bi) * p.ldy + pos : pos * p.ldy + (o0 + bi);
-      out[g] = from_f32<Tout>(tile[bi * p.pitch + q]);
+      __stcs(out + g, from_f32<Tout>(tile[bi * p.pitch + q]));
     }
   }
 }

@@ -226,9 +226,9 @@ cudaError_t launch_cols_full(int logm, int dt_in, int dt_out, const ColArgs& a, 
 // ---------------------------------------------------------------------------
 // Column transform for 1024 <= m <= 8192 with thread-block clusters.
 //
-// A cluster of CL = m / 1024 CTAs owns a strip of 32 adjacent columns over
+// A cluster of CL = m / 1024 CTAs owns a strip of 16 adjacent columns over
 // all m rows; CTA c of the cluster holds rows [1024 c, 1024 c + 1024) of the
-// strip (128 KB fp32).  Row segments are 32 columns wide (64 B bf16 / 128 B
+// strip (64 KB fp32).  Row segments are 16 columns wide (32 B bf16 / 64 B
 // fp32), so global accesses are whole sectors.  Within a CTA a thread owns
 // one 4-column quad and 32 rows: first rows tr + 32k (the register bits are
 // row bits 5..9), then, after one pass through shared memory, rows
@@ -237,16 +237,25 @@ cudaError_t launch_cols_full(int logm, int dt_in, int dt_out, const ColArgs& a, 
 // vectors of one (row, quad) position from the cluster's CTAs, runs the
 // remaining log2(CL) stages and writes the CL output rows.
 // ---------------------------------------------------------------------------
+// Strip width 16 columns (4 quads): whole 32-byte sectors for bf16 rows, 64 KB
+// of shared memory and 128 threads per CTA, so three CTAs share an SM and
+// their load, exchange and store phases overlap.
+constexpr int kQuads = 4;
+constexpr int kClusterThreads = kQuads * 32;
+// 16-byte chunk of (row, quad); bit 2 is xor-ed with row bit 5 so that rows
+// 32 apart (the phase-2 pattern) fall in different bank groups.
+__device__ __forceinline__ int cs_idx(int row, int q) { return (row * kQuads + q) ^ (((row >> 5) & 1) << 2); }
+
 template <int CL, typename Tin, typename Tout>
-__global__ void __launch_bounds__(256, 1) k_cols_cluster(const ColArgs a) {
-  extern __shared__ float4 cs_smem[];  // [1024 rows][8 quads]
+__global__ void __launch_bounds__(kClusterThreads) k_cols_cluster(const ColArgs a) {
+  extern __shared__ float4 cs_smem[];  // [1024 rows][kQuads quads]
   namespace cg = cooperative_groups;
   cg::cluster_group cluster = cg::this_cluster();
   const int crank = static_cast<int>(cluster.block_rank());
-  const int64_t col0 = (int64_t(blockIdx.x) / CL) * 32;
+  const int64_t col0 = (int64_t(blockIdx.x) / CL) * (4 * kQuads);
   const int tid = threadIdx.x;
-  const int q = tid & 7;    // column quad within the strip
-  const int tr = tid >> 3;  // 0..31
+  const int q = tid % kQuads;  // column quad within the strip
+  const int tr = tid / kQuads;  // 0..31
   const int64_t row_base = int64_t(crank) * 1024;
   float x[128];
   // phase 1: rows tr + 32 k of this CTA's block
@@ -271,19 +280,19 @@ __global__ void __launch_bounds__(256, 1) k_cols_cluster(const ColArgs a) {
   reg_stages<128, 2, 7>(x);  // row bits 5..9
 #pragma unroll
   for (int k = 0; k < 32; ++k)
-    cs_smem[(tr + 32 * k) * 8 + q] = make_float4(x[4 * k], x[4 * k + 1], x[4 * k + 2], x[4 * k + 3]);
+    cs_smem[cs_idx(tr + 32 * k, q)] = make_float4(x[4 * k], x[4 * k + 1], x[4 * k + 2], x[4 * k + 3]);
   __syncthreads();
   // phase 2: rows 32 tr + r
 #pragma unroll
   for (int r = 0; r < 32; ++r) {
-    const float4 v = cs_smem[(32 * tr + r) * 8 + q];
+    const float4 v = cs_smem[cs_idx(32 * tr + r, q)];
     x[4 * r] = v.x; x[4 * r + 1] = v.y; x[4 * r + 2] = v.z; x[4 * r + 3] = v.w;
   }
   reg_stages<128, 2, 7>(x);  // row bits 0..4
   __syncthreads();           // every phase-2 read is done before the writes
 #pragma unroll
   for (int r = 0; r < 32; ++r)
-    cs_smem[(32 * tr + r) * 8 + q] = make_float4(x[4 * r], x[4 * r + 1], x[4 * r + 2], x[4 * r + 3]);
+    cs_smem[cs_idx(32 * tr + r, q)] = make_float4(x[4 * r], x[4 * r + 1], x[4 * r + 2], x[4 * r + 3]);
   cluster.sync();  // all blocks of the strip are in shared memory
   // phase 3: this CTA combines rows (c', row_low) for row_low in its share
   Tout* dst = static_cast<Tout*>(a.y) + col0 + 4 * q;
@@ -295,7 +304,7 @@ __global__ void __launch_bounds__(256, 1) k_cols_cluster(const ColArgs a) {
 #pragma unroll
     for (int c = 0; c < CL; ++c) {
       const float4* rem = cluster.map_shared_rank(cs_smem, c);
-      const float4 w = rem[row_low * 8 + q];
+      const float4 w = rem[cs_idx(row_low, q)];
       v[4 * c] = w.x; v[4 * c + 1] = w.y; v[4 * c + 2] = w.z; v[4 * c + 3] = w.w;
     }
     if constexpr (CL > 1) reg_stages<4 * CL, 2, 2 + (CL == 2 ? 1 : (CL == 4 ? 2 : 3))>(v);
@@ -319,14 +328,14 @@ __global__ void __launch_bounds__(256, 1) k_cols_cluster(const ColArgs a) {
 template <int CL, typename Tin, typename Tout>
 static cudaError_t launch_cluster_t(const ColArgs& a, cudaStream_t st) {
   auto kern = k_cols_cluster<CL, Tin, Tout>;
-  constexpr size_t smem = size_t(1024) * 8 * sizeof(float4);
+  constexpr size_t smem = size_t(1024) * kQuads * sizeof(float4);
   static std::atomic<unsigned long long> done{0};
   cudaError_t e = set_smem_attr(kern, smem, done);
   if (e != cudaSuccess) return e;
-  const int64_t strips = a.cols / 32;
+  const int64_t strips = a.cols / (4 * kQuads);
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = dim3(static_cast<unsigned>(strips * CL));
-  cfg.blockDim = dim3(256);
+  cfg.blockDim = dim3(kClusterThreads);
   cfg.dynamicSmemBytes = smem;
   cfg.stream = st;
   cudaLaunchAttribute attr[1];
@@ -350,7 +359,7 @@ static cudaError_t launch_cluster_cl(int dt_in, int dt_out, const ColArgs& a, cu
 }
 
 cudaError_t launch_cols_cluster(int logm, int dt_in, int dt_out, const ColArgs& a, cudaStream_t st) {
-  if (a.cols % 32 != 0 || a.cols / 32 > 0x7fffffffLL / 8) return cudaErrorInvalidValue;
+  if (a.cols % (4 * kQuads) != 0 || a.cols / (4 * kQuads) > 0x7fffffffLL / 8) return cudaErrorInvalidValue;
   switch (logm) {
     case 10: return launch_cluster_cl<1>(dt_in, dt_out, a, st);
     case 11: return launch_cluster_cl<2>(dt_in, dt_out, a, st);
