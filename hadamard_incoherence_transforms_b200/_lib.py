@@ -30,6 +30,7 @@ SIGNATURES = {
     "rht_quantize_pack": (_i32, [_vp, _i64, _i64, _i64, _i32, _vp, _vp, _i32, _i32, _vp, _vp, _vp, _sz, _vp]),
     "dequant_inverse": (_i32, [_vp, _vp, _i64, _i64, _i32, _i32, _vp, _vp, _vp, _i64, _i32, _vp, _sz, _vp]),
     "wht_expand_sparse": (_i32, [_vp, _vp, _i64, _i64, _i64, _i32, ctypes.c_float, _vp, _i32, _vp]),
+    "rht_quantize_pack_noalloc": (_i32, [_vp, _i64, _i64, _i64, _i32, _vp, _vp, _i32, _i32, _vp, _vp, _vp]),
 }
 
 _lib = None

@@ -190,6 +190,10 @@ int rht_impl(bool inverse, const void* x, void* y, int64_t rows, int64_t n, int6
 
 }  // namespace
 
+namespace hit {
+void set_last_error(const char* msg) { g_last_error = msg; }
+}  // namespace hit
+
 // Plan one butterfly pass applying stages order[0..cnt) (consecutive digits).
 static bool plan_pass(const int* order, int cnt, const int32_t* radices, const int64_t* S, const float* const* blocks,
                       const int64_t* n_groups, int64_t len, int64_t outer, int axis, bool transpose,

@@ -30,6 +30,9 @@ struct RowArgs {
   float sp_scale = 1.0f;
 };
 
+// Record the message hit_last_error() returns on this host thread.
+void set_last_error(const char* msg);
+
 // dtype codes (same values as the C ABI)
 enum { DT_F32 = 0, DT_BF16 = 1 };
 

@@ -186,6 +186,36 @@ HIT_API int dequant_inverse(const uint8_t* codes, const float* scales, int64_t r
 HIT_API int wht_expand_sparse(float* values, const int32_t* cols, int64_t batch, int64_t rows, int64_t n,
                       int32_t nnz, float scale, float* dense, int mode, void* stream);
 
+/*
+ * Fused RHT + group quantization without any allocation (no counterpart in
+ * the pages; a deployment convenience).
+ *
+ * Same arguments and results as rht_quantize_pack, minus the workspace.  Some
+ * callers cannot call cudaMalloc at all -- for example plug-ins whose host
+ * application owns every byte of device memory, or latency-critical paths that
+ * must never block on the allocator -- and so cannot hand the two-sided
+ * quantizer its fp32 intermediate.  This entry point places that intermediate
+ * in a scratch array the library carries as a static device variable of
+ * HIT_NOALLOC_MAX_ELEMS fp32 elements (16 MiB); every GPU that loads
+ * libhit.so holds it until the process exits.
+ *  - Two-sided calls need rows * n <= HIT_NOALLOC_MAX_ELEMS; larger problems
+ *    return HIT_EWORKSPACE.  One-sided calls (col_signs == NULL) use no
+ *    scratch and have no extra limit.
+ *  - The first two-sided call on a device resolves the array's device address
+ *    (cudaGetSymbolAddress, with that device current); make that first call
+ *    before any stream capture.
+ *  - Every call on a device shares the one array and it keeps the last call's
+ *    contents (each call overwrites all of the part it reads, so nothing needs
+ *    clearing).  Calls whose executions overlap on the GPU -- on different
+ *    streams, or from several host threads -- race on the array.
+ *  - The call allocates nothing: no cudaMalloc, cudaFree or allocating library
+ *    routine.
+ */
+#define HIT_NOALLOC_MAX_ELEMS 4194304
+HIT_API int rht_quantize_pack_noalloc(const void* x, int64_t rows, int64_t n, int64_t ldx, int dtype_in,
+                                      const int8_t* row_signs, const int8_t* col_signs, int bits, int group,
+                                      uint8_t* codes, float* scales, void* stream);
+
 #ifdef __cplusplus
 }
 #endif
