@@ -211,10 +211,14 @@ static bool plan_pass(const int* order, int cnt, const int32_t* radices, const i
   const size_t budget = 100 * 1024;  // two CTAs per SM overlap their load / compute / store phases
   // consecutive lo values per tile (a power of two dividing S_in); along rows
   // they are contiguous in memory, so up to eight of them per tile
-  int log_nl = 0;
+  int max_nl = 0;
   if (axis == 1)
-    while (log_nl < 3 && S_in % (int64_t(2) << log_nl) == 0) ++log_nl;
-  for (; log_nl >= 0; --log_nl) {
+    while (max_nl < 3 && S_in % (int64_t(2) << max_nl) == 0) ++max_nl;
+  // Among the (NL, NB) that fit, take the largest tile (fewest chunks and
+  // barriers per element); on ties prefer more contiguous lo values.
+  int best_nl = -1, best_nb = -1;
+  int64_t best_elems = 0, best_blk = 0, best_pitch = 0;
+  for (int log_nl = max_nl; log_nl >= 0; --log_nl) {
     const int NL = 1 << log_nl;
     int64_t blk = 0;
     for (int k = 0; k < cnt; ++k) {
@@ -225,47 +229,56 @@ static bool plan_pass(const int* order, int cnt, const int32_t* radices, const i
     }
     const int64_t pnl = P * NL;
     const int64_t pitch = (pnl % 2 == 0) ? pnl + 1 : pnl;
-    for (int log_nb = 6; log_nb >= 0; --log_nb) {
-      const int nb = 1 << log_nb;
+    for (int log_nb = 8; log_nb >= 0; --log_nb) {
+      const int64_t nb = int64_t(1) << log_nb;
       const size_t bytes = static_cast<size_t>(blk + nb * pitch) * sizeof(float);
-      if (bytes > budget) continue;
-      p = hit::BflyPass();
-      p.outer = outer;
-      p.axis = axis;
-      p.P = static_cast<int>(P);
-      p.S_in = S_in;
-      p.NL = NL;
-      p.log_nl = log_nl;
-      p.NB = nb;
-      p.log_nb = log_nb;
-      p.div_pnl = hit::make_fastdiv(static_cast<uint32_t>(pnl));
-      p.pitch = static_cast<int>(pitch);
-      p.n_tiles = (len / (P * S_in)) * (S_in / NL);
-      p.blk_floats = static_cast<int>(blk);
-      p.ns = cnt;
-      int ofs = 0;
-      for (int k = 0; k < cnt; ++k) {
-        const int t = order[k];
-        hit::BflyStage& st = p.st[k];
-        st.blocks = blocks[t];
-        st.b = radices[t];
-        st.bp = (st.b + 3) / 4 * 4;
-        st.ls = static_cast<int>(S[t] / S_in);
-        st.div_ls = hit::make_fastdiv(static_cast<uint32_t>(st.ls));
-        st.sofs = ofs;
-        st.shared_block = (n_groups[t] == 1 && len / radices[t] != 1) ? 1 : 0;
-        st.transpose = transpose ? 1 : 0;
-        ofs += (st.shared_block ? 1 : static_cast<int>((P / st.b) * NL)) * st.b * st.bp;
+      if (bytes > budget || nb * pnl > 32768) continue;
+      if (nb * pnl > best_elems) {
+        best_elems = nb * pnl;
+        best_nl = log_nl;
+        best_nb = log_nb;
+        best_blk = blk;
+        best_pitch = pitch;
       }
-      // enough CTAs to fill the machine a few times over
-      const int64_t chunks = (outer + nb - 1) / nb;
-      int64_t splits = (4 * 148 + p.n_tiles - 1) / p.n_tiles;
-      splits = splits < 1 ? 1 : (splits > chunks ? chunks : splits);
-      p.chunks_per_split = (chunks + splits - 1) / splits;
-      return true;
+      break;  // smaller NB only shrinks the tile for this NL
     }
   }
-  return false;
+  if (best_nl < 0) return false;
+  const int NL = 1 << best_nl, nb = 1 << best_nb;
+  p = hit::BflyPass();
+  p.outer = outer;
+  p.axis = axis;
+  p.P = static_cast<int>(P);
+  p.S_in = S_in;
+  p.NL = NL;
+  p.log_nl = best_nl;
+  p.NB = nb;
+  p.log_nb = best_nb;
+  p.div_pnl = hit::make_fastdiv(static_cast<uint32_t>(P * NL));
+  p.pitch = static_cast<int>(best_pitch);
+  p.n_tiles = (len / (P * S_in)) * (S_in / NL);
+  p.blk_floats = static_cast<int>(best_blk);
+  p.ns = cnt;
+  int ofs = 0;
+  for (int k = 0; k < cnt; ++k) {
+    const int t = order[k];
+    hit::BflyStage& st = p.st[k];
+    st.blocks = blocks[t];
+    st.b = radices[t];
+    st.bp = (st.b + 3) / 4 * 4;
+    st.ls = static_cast<int>(S[t] / S_in);
+    st.div_ls = hit::make_fastdiv(static_cast<uint32_t>(st.ls));
+    st.sofs = ofs;
+    st.shared_block = (n_groups[t] == 1 && len / radices[t] != 1) ? 1 : 0;
+    st.transpose = transpose ? 1 : 0;
+    ofs += (st.shared_block ? 1 : static_cast<int>((P / st.b) * NL)) * st.b * st.bp;
+  }
+  // enough CTAs to fill the machine a few times over
+  const int64_t chunks = (outer + nb - 1) / nb;
+  int64_t splits = (4 * 148 + p.n_tiles - 1) / p.n_tiles;
+  splits = splits < 1 ? 1 : (splits > chunks ? chunks : splits);
+  p.chunks_per_split = (chunks + splits - 1) / splits;
+  return true;
 }
 
 extern "C" {

@@ -19,11 +19,11 @@ namespace hit {
 
 __device__ unsigned int g_wait_timeouts = 0;
 
-// Warps per CTA: one producer plus consumers.  Seven warps keep at most two
-// warps per SM sub-partition, which leaves each thread the full 255 registers
-// for its row elements.
+// Warps per CTA: one producer plus consumers.  Eight warps keep two warps per
+// SM sub-partition, which leaves each thread the full 255 registers for its
+// row elements.
 #ifndef HIT_STREAM_WARPS
-#define HIT_STREAM_WARPS 7
+#define HIT_STREAM_WARPS 8
 #endif
 
 // Ring protocol.  Row k of this CTA goes to slot k % S and is consumed by team
