@@ -10,18 +10,22 @@ namespace hit {
 // Group-wise symmetric absmax round-to-nearest, in layout B.
 //
 // Per group: a = max|y|, s = a / qmax (IEEE division), q = rint(y / s) with
-// ties to even, stored code u = q + 2^(bits-1).  The division per element is
-// replaced by a multiply with r = 1/s (correctly rounded reciprocal): the
-// exact product y*r differs from the quotient y/s by at most |y/s| * 2^-24 and
-// fl(y/s) from y/s by half an ulp, together < 7e-7 for |y/s| <= qmax <= 7.  So
-// whenever y*r is more than 2^-18 away from a half-integer, fl(y/s) and y*r
-// round to the same integer and the fast result equals rint(fl(y/s)).  A
-// 32-element chunk holding any element inside that margin (probability about
-// 1e-5 per element) is redone with correctly rounded division.  The fast
-// integer comes from fma(y, r, 1.5*2^23 + 2^(bits-1)): that sum lies in
-// [2^23, 2^24) where the float spacing is 1, so its bit pattern is
-// 0x4B400000 + u and the low byte is the stored code.  |y*r| <= a*r <=
-// qmax*(1 + 2^-22) < qmax + 1/2, so the fast path never needs a clamp.
+// ties to even, stored code u = q + 2^(bits-1).
+//
+// The quotient t = RN(y / s) is computed without a divide instruction by
+// Markstein's correction step (P. Markstein, "Computation of elementary
+// functions on the IBM RISC System/6000 processor", IBM J. Res. Dev. 34(1),
+// 1990): with r = RN(1/s) and q0 = RN(y r) (within one ulp of y/s), the
+// remainder e = y - s q0 is exact in one fma and RN(q0 + e r) is the
+// correctly rounded quotient, barring underflow and overflow.  Groups whose
+// scale lies outside [2^-100, 2^100] are rescaled by an exact power of two
+// first (y/s is unchanged; elements that underflow in the rescale have
+// |y/s| far below 1/2 and quantize to 0 either way).  Every element is then
+// rounded to an integer by adding 1.5*2^23 + 2^(bits-1): the sum lies in
+// [2^23, 2^24) where the float spacing is 1, so the add rounds t to the
+// nearest integer with ties to even (the offset is even) and the low byte of
+// the sum's bit pattern is the stored code.  |t| <= qmax (1 + 2^-23), so no
+// clamp is needed.  The fp32 operations are packed two per instruction.
 //
 // When log2(n) is even, 1/sqrt(n) is a power of two and is folded exactly
 // into the scale: y = acc * 2^-k, s = s_acc * 2^-k, y/s = acc/s_acc.
@@ -32,13 +36,19 @@ struct QConst {
   static constexpr float MAGIC = 12582912.0f + float(1 << (BITS - 1));
 };
 
+// Codes of 32 elements of one group with scale s (s > 0) and r = RN(1/s).
 template <int BITS>
-__device__ __forceinline__ void quant_chunk_exact(const float* x, float s, uint32_t* ub) {
+__device__ __forceinline__ void quant_chunk(const float* xc, float s, float r, uint32_t* ub) {
+  constexpr float MAGIC = QConst<BITS>::MAGIC;
 #pragma unroll
-  for (int e = 0; e < 32; ++e) {
-    float q = rintf(__fdiv_rn(x[e], s));
-    q = fminf(fmaxf(q, -QConst<BITS>::QMAX), QConst<BITS>::QMAX);
-    ub[e] = __float_as_uint(q + QConst<BITS>::MAGIC);
+  for (int e = 0; e < 32; e += 2) {
+    float q0, q1, e0, e1, t0, t1, m0, m1;
+    fma_x2(xc[e], xc[e + 1], r, r, 0.0f, 0.0f, q0, q1);      // q0 = RN(y r)
+    fma_x2(q0, q1, -s, -s, xc[e], xc[e + 1], e0, e1);         // e = y - s q0 (exact)
+    fma_x2(e0, e1, r, r, q0, q1, t0, t1);                     // t = RN(q0 + e r) = RN(y / s)
+    fma_x2(t0, t1, 1.0f, 1.0f, MAGIC, MAGIC, m0, m1);         // RN(t + MAGIC) = rint(t) + MAGIC
+    ub[e] = __float_as_uint(m0);
+    ub[e + 1] = __float_as_uint(m1);
   }
 }
 
@@ -90,30 +100,25 @@ __device__ __forceinline__ void quant_rowB(float (&x)[Geom<LOGN>::E], const RowA
   constexpr int NW = E * BITS / 32;  // packed words per thread
   uint32_t W[NW];
   const int64_t spr = int64_t(G::N) >> lg;
+  float s = 0.0f, ss = 0.0f, r = 0.0f, k = 1.0f;
 #pragma unroll
   for (int cc = 0; cc < NCH; ++cc) {
-    const float s = __fdiv_rn(mx[cc], QMAX);
     const int e0 = E * tau + 32 * cc;
-    if ((e0 & ((1 << lg) - 1)) == 0) a.scales[row * spr + (e0 >> lg)] = FOLD ? s * a.norm : s;
-    const float* xc = x + 32 * cc;
+    if (cc == 0 || (e0 & ((1 << lg) - 1)) == 0) {  // first chunk of a group: its scale
+      s = __fdiv_rn(mx[cc], QMAX);
+      if ((e0 & ((1 << lg) - 1)) == 0) a.scales[row * spr + (e0 >> lg)] = FOLD ? s * a.norm : s;
+      k = s < 0x1p-100f ? 0x1p100f : (s > 0x1p100f ? 0x1p-100f : 1.0f);
+      ss = s * k;
+      r = s > 0.0f ? __frcp_rn(ss) : 0.0f;
+    }
+    float* xc = x + 32 * cc;
     uint32_t ub[32];
-    if (s >= 0x1p-125f) {
-      const float r = __frcp_rn(s);
-      // m = fl(y*r + MAGIC) (the rounded code), d = fl(y*r - (m - MAGIC)) its residual
-      float dmax = 0.0f;
+    if (s > 0.0f) {
+      if (k != 1.0f) {
 #pragma unroll
-      for (int e = 0; e < 32; e += 2) {
-        float m0, m1, n0, n1, d0, d1;
-        fma_x2(xc[e], xc[e + 1], r, r, MAGIC, MAGIC, m0, m1);
-        sub_x2(MAGIC, MAGIC, m0, m1, n0, n1);
-        fma_x2(xc[e], xc[e + 1], r, r, n0, n1, d0, d1);
-        dmax = fmaxf(dmax, fmaxf(fabsf(d0), fabsf(d1)));
-        ub[e] = __float_as_uint(m0);
-        ub[e + 1] = __float_as_uint(m1);
+        for (int e = 0; e < 32; e += 2) mul_x2(xc[e], xc[e + 1], k, k);
       }
-      if (dmax > 0.5f - 0x1p-18f) quant_chunk_exact<BITS>(xc, s, ub);
-    } else if (s > 0.0f) {
-      quant_chunk_exact<BITS>(xc, s, ub);
+      quant_chunk<BITS>(xc, ss, r, ub);
     } else {
 #pragma unroll
       for (int e = 0; e < 32; ++e) ub[e] = __float_as_uint(MAGIC);

@@ -26,13 +26,16 @@ __device__ unsigned int g_wait_timeouts = 0;
 #define HIT_STREAM_WARPS 8
 #endif
 
-// Ring protocol.  Row k of this CTA goes to slot k % S and is consumed by team
-// k % TEAMS.  S is a multiple of TEAMS, so every slot is always served by the
-// same team, which takes the slot's phases strictly in order: when a team
-// waits for phase j of a slot's "full" barrier it has itself consumed phase
-// j-1, and the producer refills a slot only after its "empty" barrier
-// completed the previous phase.  A parity wait therefore never sees a barrier
-// two phases behind or ahead of the phase it asks for.
+// Ring protocol.  The producer copies this CTA's rows k = 0, 1, 2, ... in
+// order into slot k % S, refilling a slot only after its "empty" barrier has
+// completed the previous phase.  Consumer teams take rows by ticket: a team
+// draws the next k from a shared counter when it starts a row, so tickets in
+// use are handed out in increasing order and every team holds one at a time.
+// A parity wait for row k on slot k % S could only be fooled if row k - S had
+// not been copied yet; the producer would then be stalled at some row r <= k - S
+// whose slot is held by ticket r - S, and every ticket in [r, k] would belong
+// to a team blocked on an uncopied row, i.e. S + 2 teams at least.  So any ring
+// with S >= TEAMS - 1 is safe, and the ring takes every slot that fits.
 template <int LOGN, typename Tin>
 struct StreamCfg {
   using G = Geom<LOGN>;
@@ -44,11 +47,14 @@ struct StreamCfg {
   static constexpr uint32_t ROW = uint32_t(G::N) * sizeof(Tin);
   static constexpr uint32_t SIGNS = uint32_t(G::N) * 4;        // sign-bit mask per column
   static constexpr uint32_t SMEM_MAX = 232448;                 // opt-in limit per CTA on sm_100
-  static constexpr int S = TEAMS * int((SMEM_MAX - 1024 - SIGNS) / (SLOT * TEAMS));  // ring depth
+  static constexpr int S = int((SMEM_MAX - 1024 - SIGNS) / SLOT);  // ring depth
   static constexpr size_t SMEM = 1024 + SIGNS + size_t(S) * SLOT;
   static constexpr int THREADS = (NCW + 1) * 32;
-  static_assert(TEAMS >= 1 && S >= TEAMS && S % TEAMS == 0, "ring depth must be a multiple of the team count");
-  static_assert(2 * S * 8 <= 1024, "barriers must fit in the first kilobyte");
+  static constexpr int BAR_CONSUMERS = 15;                     // named barrier of all consumer warps
+  static_assert(TEAMS >= 1 && S + 1 >= TEAMS, "ring too shallow for the ticket protocol");
+  static_assert(TEAMS + 1 < BAR_CONSUMERS, "named barrier ids");
+  static_assert(S <= 32, "the ramp issues one ring slot per producer lane");
+  static_assert(2 * S * 8 + 8 + 4 * TEAMS <= 1024, "barriers and tickets must fit in the first kilobyte");
 };
 
 template <int LOGN, typename Tin>
@@ -60,6 +66,40 @@ __device__ __forceinline__ void stream_team_sync(int team) {
   }
 }
 
+// The sign vector as sign-bit masks (0 or 0x80000000 per column), one
+// shared-memory table per CTA.  Each consumer thread loads its (at most two)
+// 16-byte pieces of the int8 signs before the producer starts its copies, so
+// these loads are not queued behind the first wave of row copies.
+template <int N, int NTHREADS>
+struct SignLoad {
+  static constexpr int PIECES = N / 16;
+  static constexpr int PER = (PIECES + NTHREADS - 1) / NTHREADS;
+  uint4 v[PER];
+  __device__ __forceinline__ void load(const int8_t* __restrict__ s, int t) {
+    if ((reinterpret_cast<uintptr_t>(s) & 15) != 0) return;  // unaligned signs: store() reads bytes
+#pragma unroll
+    for (int p = 0; p < PER; ++p)
+      if (t + p * NTHREADS < PIECES) v[p] = __ldg(reinterpret_cast<const uint4*>(s) + t + p * NTHREADS);
+  }
+  __device__ __forceinline__ void store(uint32_t* sgn, const int8_t* __restrict__ s, int t) const {
+    if ((reinterpret_cast<uintptr_t>(s) & 15) != 0) {
+      for (int i = t; i < N; i += NTHREADS) sgn[i] = s[i] < 0 ? 0x80000000u : 0u;
+      return;
+    }
+#pragma unroll
+    for (int p = 0; p < PER; ++p) {
+      const int i = t + p * NTHREADS;
+      if (i >= PIECES) break;
+      const uint32_t w[4] = {v[p].x, v[p].y, v[p].z, v[p].w};
+#pragma unroll
+      for (int k = 0; k < 4; ++k)
+        reinterpret_cast<uint4*>(sgn)[4 * i + k] =
+            make_uint4((w[k] << 24) & 0x80000000u, (w[k] << 16) & 0x80000000u, (w[k] << 8) & 0x80000000u,
+                       w[k] & 0x80000000u);
+    }
+  }
+};
+
 template <int LOGN, typename Tin, typename Tout, int EPI, int BITS>
 __global__ void __launch_bounds__(StreamCfg<LOGN, Tin>::THREADS, 1) k_rows_stream(const RowArgs a) {
   using G = Geom<LOGN>;
@@ -67,18 +107,22 @@ __global__ void __launch_bounds__(StreamCfg<LOGN, Tin>::THREADS, 1) k_rows_strea
   extern __shared__ __align__(1024) uint8_t smem[];
   uint64_t* full = reinterpret_cast<uint64_t*>(smem);
   uint64_t* empty = full + C::S;
+  int* ticket = reinterpret_cast<int*>(empty + C::S);
+  volatile int* abort = ticket + 1;
+  int* team_ticket = ticket + 2;
   uint32_t* sgn = reinterpret_cast<uint32_t*>(smem + 1024);
   uint8_t* slots = smem + 1024 + C::SIGNS;
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const bool has_signs = a.pre_signs != nullptr;
-  if (has_signs) {  // the sign vector as sign-bit masks, shared by every row of this CTA
-    for (int i = threadIdx.x; i < G::N; i += blockDim.x) sgn[i] = a.pre_signs[i] < 0 ? 0x80000000u : 0u;
-  }
+  SignLoad<G::N, C::NCW * 32> sl;
+  if (has_signs && warp < C::NCW) sl.load(a.pre_signs, threadIdx.x);
   if (threadIdx.x == 0) {
     for (int s = 0; s < C::S; ++s) {
       mbar_init(&full[s], 1);
       mbar_init(&empty[s], C::WPR);
     }
+    ticket[0] = 0;
+    ticket[1] = 0;
     mbar_init_fence();
   }
   __syncthreads();
@@ -86,18 +130,35 @@ __global__ void __launch_bounds__(StreamCfg<LOGN, Tin>::THREADS, 1) k_rows_strea
   const int64_t nrows = a.rows > blockIdx.x ? (a.rows - blockIdx.x + grid - 1) / grid : 0;
 
   if (warp == C::NCW) {  // producer
+    const uint8_t* src = static_cast<const uint8_t*>(a.x);
+    auto issue = [&](int64_t k) {
+      const int s = int(k % C::S);
+      const int64_t row = blockIdx.x + k * grid;
+      mbar_expect_tx(&full[s], C::ROW);
+      bulk_g2s(slots + size_t(s) * C::SLOT, src + row * a.ldx * int64_t(sizeof(Tin)), C::ROW, &full[s]);
+    };
+    // Ramp: one row per team from parallel lanes, the rest of the ring once
+    // the first row has landed (a smaller first wave arrives sooner).
+    const int64_t wave1 = nrows < C::TEAMS ? nrows : C::TEAMS;
+    const int64_t wave2 = nrows < C::S ? nrows : C::S;
+    if (lane < wave1) issue(lane);
+    __syncwarp();
+    bool ok = true;
+    if (wave2 > wave1) {
+      if (lane == 0) ok = mbar_wait(&full[0], 0u);
+      ok = __shfl_sync(0xffffffffu, ok, 0);
+      if (ok && lane >= wave1 && lane < wave2) issue(lane);
+      __syncwarp();
+    }
     if (lane == 0) {
-      const uint8_t* src = static_cast<const uint8_t*>(a.x);
-      int64_t issued = 0;
-      for (int64_t k = 0; k < nrows; ++k) {
-        const int s = int(k % C::S);
-        if (k >= C::S && !mbar_wait(&empty[s], uint32_t((k / C::S) - 1) & 1u)) {
+      int64_t issued = ok ? wave2 : wave1;
+      if (!ok) atomicAdd(&g_wait_timeouts, 1u);
+      for (int64_t k = issued; ok && k < nrows; ++k) {
+        if (!mbar_wait(&empty[k % C::S], uint32_t((k / C::S) - 1) & 1u)) {
           atomicAdd(&g_wait_timeouts, 1u);
           break;
         }
-        const int64_t row = blockIdx.x + k * grid;
-        mbar_expect_tx(&full[s], C::ROW);
-        bulk_g2s(slots + size_t(s) * C::SLOT, src + row * a.ldx * int64_t(sizeof(Tin)), C::ROW, &full[s]);
+        issue(k);
         issued = k + 1;
       }
       // Do not leave while a copy into this CTA's shared memory is in flight.
@@ -107,13 +168,34 @@ __global__ void __launch_bounds__(StreamCfg<LOGN, Tin>::THREADS, 1) k_rows_strea
     return;
   }
 
+  if (has_signs) {
+    sl.store(sgn, a.pre_signs, threadIdx.x);
+    asm volatile("bar.sync %0, %1;" ::"r"(C::BAR_CONSUMERS), "r"(C::NCW * 32) : "memory");
+  }
   const int team = warp / C::WPR;
   const int tau = (warp % C::WPR) * 32 + lane;
-  for (int64_t k = team; k < nrows; k += C::TEAMS) {
+  for (;;) {
+    int64_t k;
+    if constexpr (C::WPR == 1) {
+      int t = 0;
+      if (lane == 0) t = atomicAdd(ticket, 1);
+      k = __shfl_sync(0xffffffffu, t, 0);
+    } else {
+      // The leader's write for the next row comes after this row's two team
+      // barriers, so the partner warp has read this value by then.
+      if (tau == 0) team_ticket[team] = atomicAdd(ticket, 1);
+      stream_team_sync<LOGN, Tin>(team);
+      k = *abort ? nrows : team_ticket[team];
+    }
+    if (k >= nrows) break;
     const int s = int(k % C::S);
     if (!mbar_wait(&full[s], uint32_t(k / C::S) & 1u)) {
       if (lane == 0) atomicAdd(&g_wait_timeouts, 1u);
-      return;
+      // A one-warp team stops here.  A two-warp team finishes the row (its
+      // partner is at the same team barriers) and both warps stop at the next
+      // ticket; the row's output is then undefined and the counter says so.
+      if constexpr (C::WPR == 1) return;
+      *abort = 1;
     }
     const int64_t row = blockIdx.x + k * grid;
     uint8_t* slot = slots + size_t(s) * C::SLOT;
