@@ -66,10 +66,11 @@ int check_rows_operand(const void* p, int64_t ld, int64_t n, int dt, const char*
   return HIT_OK;
 }
 
-// Rows of 4096 or 8192 elements go through the persistent TMA-fed kernel; its
-// bulk copies need 16-byte aligned row starts (always true for the row
-// pitches the checks accept when n >= 4096).
-bool use_stream(int logn, const void* x, int64_t ld, int dt) {
+// Rows of 4096 elements go through the persistent TMA-fed kernel, rows of
+// 8192 through the persistent direct-load kernel; both need 16-byte aligned
+// row starts (always true for the row pitches the checks accept when
+// n >= 4096 and the base is 16-byte aligned).
+bool use_persistent(int logn, const void* x, int64_t ld, int dt) {
   return (logn == 12 || logn == 13) && aligned(x, 16) && (static_cast<size_t>(ld) * esize(dt)) % 16 == 0;
 }
 
@@ -163,7 +164,8 @@ int rht_impl(bool inverse, const void* x, void* y, int64_t rows, int64_t n, int6
     a.norm = inv_sqrt(n);
     const int logn = ilog2(n);
     cudaError_t e;
-    if (use_stream(logn, x, ldx, dt_in)) e = hit::rows_stream_store(logn, dt_in, dt_out, a, st);
+    if (use_persistent(logn, x, ldx, dt_in))
+      e = logn == 12 ? hit::rows_stream_store(logn, dt_in, dt_out, a, st) : hit::rows_direct_store(logn, dt_in, dt_out, a, st);
     else if (dt_in == HIT_F32) e = hit::rows_store_from_f32(logn, dt_out, a, st);
     else e = hit::rows_store_from_bf16(logn, dt_out, a, st);
     return cuda_status(e, fn);
@@ -472,7 +474,8 @@ int rht_quantize_pack(const void* x, int64_t rows, int64_t n, int64_t ldx, int d
   }
   const int logn = ilog2(n);
   cudaError_t e;
-  if (use_stream(logn, a.x, a.ldx, dt_rows)) e = hit::rows_stream_quant(logn, dt_rows, bits, a, st);
+  if (use_persistent(logn, a.x, a.ldx, dt_rows))
+    e = logn == 12 ? hit::rows_stream_quant(logn, dt_rows, bits, a, st) : hit::rows_direct_quant(logn, dt_rows, bits, a, st);
   else if (bits == 4) e = hit::rows_quant_b4(logn, dt_rows, a, st);
   else if (bits == 3) e = hit::rows_quant_b3(logn, dt_rows, a, st);
   else e = hit::rows_quant_b2(logn, dt_rows, a, st);

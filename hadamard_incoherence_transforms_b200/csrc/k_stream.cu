@@ -1,33 +1,28 @@
-// Persistent TMA-fed row kernels for n = 4096 and 8192 (see rows_stream.cuh).
+// Persistent TMA-fed row kernels for n = 4096 (see rows_stream.cuh).
 #include "kernels.h"
 #include "rows_stream.cuh"
 
 namespace hit {
 
 template <typename Tin>
-static cudaError_t quant_logn(int logn, int bits, const RowArgs& a, cudaStream_t st) {
-  if (logn == 12) {
-    if (bits == 4) return launch_stream<12, Tin, float, EPI_QUANT, 4>(a, st);
-    if (bits == 3) return launch_stream<12, Tin, float, EPI_QUANT, 3>(a, st);
-    return launch_stream<12, Tin, float, EPI_QUANT, 2>(a, st);
-  }
-  if (bits == 4) return launch_stream<13, Tin, float, EPI_QUANT, 4>(a, st);
-  if (bits == 3) return launch_stream<13, Tin, float, EPI_QUANT, 3>(a, st);
-  return launch_stream<13, Tin, float, EPI_QUANT, 2>(a, st);
+static cudaError_t quant_bits(int bits, const RowArgs& a, cudaStream_t st) {
+  if (bits == 4) return launch_stream<12, Tin, float, EPI_QUANT, 4>(a, st);
+  if (bits == 3) return launch_stream<12, Tin, float, EPI_QUANT, 3>(a, st);
+  return launch_stream<12, Tin, float, EPI_QUANT, 2>(a, st);
 }
 
 cudaError_t rows_stream_quant(int logn, int dt_in, int bits, const RowArgs& a, cudaStream_t st) {
-  if (logn != 12 && logn != 13) return cudaErrorInvalidValue;
-  return dt_in == DT_F32 ? quant_logn<float>(logn, bits, a, st) : quant_logn<__nv_bfloat16>(logn, bits, a, st);
+  if (logn != 12) return cudaErrorInvalidValue;
+  return dt_in == DT_F32 ? quant_bits<float>(bits, a, st) : quant_bits<__nv_bfloat16>(bits, a, st);
 }
 
 template <typename Tin, typename Tout>
 static cudaError_t store_logn(int logn, const RowArgs& a, cudaStream_t st) {
-  return logn == 12 ? launch_stream<12, Tin, Tout, EPI_STORE, 0>(a, st) : launch_stream<13, Tin, Tout, EPI_STORE, 0>(a, st);
+  return launch_stream<12, Tin, Tout, EPI_STORE, 0>(a, st);
 }
 
 cudaError_t rows_stream_store(int logn, int dt_in, int dt_out, const RowArgs& a, cudaStream_t st) {
-  if (logn != 12 && logn != 13) return cudaErrorInvalidValue;
+  if (logn != 12) return cudaErrorInvalidValue;
   if (dt_in == DT_F32) return dt_out == DT_F32 ? store_logn<float, float>(logn, a, st) : store_logn<float, __nv_bfloat16>(logn, a, st);
   return dt_out == DT_F32 ? store_logn<__nv_bfloat16, float>(logn, a, st)
                           : store_logn<__nv_bfloat16, __nv_bfloat16>(logn, a, st);

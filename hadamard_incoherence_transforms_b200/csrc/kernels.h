@@ -16,4 +16,7 @@ cudaError_t rows_sparse_all(int logn, int mode, const RowArgs& a, cudaStream_t s
 cudaError_t rows_stream_quant(int logn, int dt_in, int bits, const RowArgs& a, cudaStream_t st);
 cudaError_t rows_stream_store(int logn, int dt_in, int dt_out, const RowArgs& a, cudaStream_t st);
 unsigned int read_wait_timeouts();
+// Persistent direct-load variants for n = 4096 / 8192.
+cudaError_t rows_direct_quant(int logn, int dt_in, int bits, const RowArgs& a, cudaStream_t st);
+cudaError_t rows_direct_store(int logn, int dt_in, int dt_out, const RowArgs& a, cudaStream_t st);
 }  // namespace hit

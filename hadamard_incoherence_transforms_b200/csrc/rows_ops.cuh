@@ -36,12 +36,14 @@ struct QConst {
   static constexpr float MAGIC = 12582912.0f + float(1 << (BITS - 1));
 };
 
-// Codes of 32 elements of one group with scale s (s > 0) and r = RN(1/s).
+// Codes of 8 elements of one group with scale s and r = RN(1/s).  An all-zero
+// group passes r = 0 (and s = 1): every quotient is then 0 and the code is
+// the offset 2^(bits-1).
 template <int BITS>
-__device__ __forceinline__ void quant_chunk(const float* xc, float s, float r, uint32_t* ub) {
+__device__ __forceinline__ void quant8(const float* xc, float s, float r, uint32_t* ub) {
   constexpr float MAGIC = QConst<BITS>::MAGIC;
 #pragma unroll
-  for (int e = 0; e < 32; e += 2) {
+  for (int e = 0; e < 8; e += 2) {
     float q0, q1, e0, e1, t0, t1, m0, m1;
     fma_x2(xc[e], xc[e + 1], r, r, 0.0f, 0.0f, q0, q1);      // q0 = RN(y r)
     fma_x2(q0, q1, -s, -s, xc[e], xc[e + 1], e0, e1);         // e = y - s q0 (exact)
@@ -52,8 +54,11 @@ __device__ __forceinline__ void quant_chunk(const float* xc, float s, float r, u
   }
 }
 
-template <int LOGN, int BITS>
-__device__ __forceinline__ void quant_rowB(float (&x)[Geom<LOGN>::E], const RowArgs& a, int64_t row, int tau) {
+// next(cc) runs after chunk cc's values are consumed; a persistent kernel uses
+// it to refill x[32cc .. 32cc+31] with its next row.
+template <int LOGN, int BITS, typename Next>
+__device__ __forceinline__ void quant_rowB_next(float (&x)[Geom<LOGN>::E], const RowArgs& a, int64_t row, int tau,
+                                                Next&& next) {
   using G = Geom<LOGN>;
   constexpr int E = G::E;
   constexpr int NCH = E / 32;
@@ -97,8 +102,13 @@ __device__ __forceinline__ void quant_rowB(float (&x)[Geom<LOGN>::E], const RowA
     for (int cc = 0; cc < NCH; ++cc) mx[cc] = m;
   }
 
+  // 4- and 2-bit codes are packed and stored one 32-element chunk at a time
+  // (16 or 8 bytes per chunk); 3-bit chunks (12 bytes) are collected and
+  // stored as 16-byte vectors at the end.
   constexpr int NW = E * BITS / 32;  // packed words per thread
-  uint32_t W[NW];
+  constexpr int CW = BITS;           // packed words per 32-element chunk
+  uint32_t W[BITS == 3 ? NW : 1];
+  uint8_t* dst = a.codes + row * (int64_t(G::N) * BITS / 8) + int64_t(tau) * (E * BITS / 8);
   const int64_t spr = int64_t(G::N) >> lg;
   float s = 0.0f, ss = 0.0f, r = 0.0f, k = 1.0f;
 #pragma unroll
@@ -112,39 +122,54 @@ __device__ __forceinline__ void quant_rowB(float (&x)[Geom<LOGN>::E], const RowA
       r = s > 0.0f ? __frcp_rn(ss) : 0.0f;
     }
     float* xc = x + 32 * cc;
-    uint32_t ub[32];
-    if (s > 0.0f) {
-      if (k != 1.0f) {
+    if (k != 1.0f) {
 #pragma unroll
-        for (int e = 0; e < 32; e += 2) mul_x2(xc[e], xc[e + 1], k, k);
-      }
-      quant_chunk<BITS>(xc, ss, r, ub);
-    } else {
-#pragma unroll
-      for (int e = 0; e < 32; ++e) ub[e] = __float_as_uint(MAGIC);
+      for (int e = 0; e < 32; e += 2) mul_x2(xc[e], xc[e + 1], k, k);
     }
+    const float rr = s > 0.0f ? r : 0.0f;
+    const float sx = s > 0.0f ? ss : 1.0f;
     if constexpr (BITS == 4) {
+      uint32_t w[4];
 #pragma unroll
-      for (int w = 0; w < 4; ++w) W[4 * cc + w] = pack4x8(ub + 8 * w);
+      for (int v = 0; v < 4; ++v) {
+        uint32_t ub[8];
+        quant8<BITS>(xc + 8 * v, sx, rr, ub);
+        w[v] = pack4x8(ub);
+      }
+      __stcs(reinterpret_cast<uint4*>(dst) + cc, make_uint4(w[0], w[1], w[2], w[3]));
     } else if constexpr (BITS == 2) {
+      uint32_t w[2];
 #pragma unroll
-      for (int w = 0; w < 2; ++w) W[2 * cc + w] = pack2x16(ub + 16 * w);
+      for (int v = 0; v < 2; ++v) {
+        uint32_t ub[16];
+        quant8<BITS>(xc + 16 * v, sx, rr, ub);
+        quant8<BITS>(xc + 16 * v + 8, sx, rr, ub + 8);
+        w[v] = pack2x16(ub);
+      }
+      __stcs(reinterpret_cast<uint2*>(dst) + cc, make_uint2(w[0], w[1]));
     } else {
-      pack3x32(ub, W + 3 * cc);
+      uint32_t ub[32];
+#pragma unroll
+      for (int v = 0; v < 4; ++v) quant8<BITS>(xc + 8 * v, sx, rr, ub + 8 * v);
+      pack3x32(ub, W + CW * cc);
+    }
+    next(cc);
+  }
+  if constexpr (BITS == 3) {
+    if constexpr (NW % 4 == 0) {
+#pragma unroll
+      for (int v = 0; v < NW / 4; ++v)
+        __stcs(reinterpret_cast<uint4*>(dst) + v, make_uint4(W[4 * v], W[4 * v + 1], W[4 * v + 2], W[4 * v + 3]));
+    } else {
+#pragma unroll
+      for (int v = 0; v < NW; ++v) __stcs(reinterpret_cast<uint32_t*>(dst) + v, W[v]);
     }
   }
-  uint8_t* dst = a.codes + row * (int64_t(G::N) * BITS / 8) + int64_t(tau) * (E * BITS / 8);
-  if constexpr (NW % 4 == 0) {
-#pragma unroll
-    for (int v = 0; v < NW / 4; ++v)
-      __stcs(reinterpret_cast<uint4*>(dst) + v, make_uint4(W[4 * v], W[4 * v + 1], W[4 * v + 2], W[4 * v + 3]));
-  } else if constexpr (NW % 2 == 0) {
-#pragma unroll
-    for (int v = 0; v < NW / 2; ++v) __stcs(reinterpret_cast<uint2*>(dst) + v, make_uint2(W[2 * v], W[2 * v + 1]));
-  } else {
-#pragma unroll
-    for (int v = 0; v < NW; ++v) __stcs(reinterpret_cast<uint32_t*>(dst) + v, W[v]);
-  }
+}
+
+template <int LOGN, int BITS>
+__device__ __forceinline__ void quant_rowB(float (&x)[Geom<LOGN>::E], const RowArgs& a, int64_t row, int tau) {
+  quant_rowB_next<LOGN, BITS>(x, a, row, tau, [](int) {});
 }
 
 // Dequantization into layout B: yhat = (u - 2^(bits-1)) * s, with the

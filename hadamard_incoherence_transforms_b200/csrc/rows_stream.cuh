@@ -100,7 +100,7 @@ struct SignLoad {
   }
 };
 
-template <int LOGN, typename Tin, typename Tout, int EPI, int BITS>
+template <int LOGN, typename Tin, typename Tout, int EPI, int BITS, bool SIGNS>
 __global__ void __launch_bounds__(StreamCfg<LOGN, Tin>::THREADS, 1) k_rows_stream(const RowArgs a) {
   using G = Geom<LOGN>;
   using C = StreamCfg<LOGN, Tin>;
@@ -113,9 +113,8 @@ __global__ void __launch_bounds__(StreamCfg<LOGN, Tin>::THREADS, 1) k_rows_strea
   uint32_t* sgn = reinterpret_cast<uint32_t*>(smem + 1024);
   uint8_t* slots = smem + 1024 + C::SIGNS;
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const bool has_signs = a.pre_signs != nullptr;
   SignLoad<G::N, C::NCW * 32> sl;
-  if (has_signs && warp < C::NCW) sl.load(a.pre_signs, threadIdx.x);
+  if (SIGNS && warp < C::NCW) sl.load(a.pre_signs, threadIdx.x);
   if (threadIdx.x == 0) {
     for (int s = 0; s < C::S; ++s) {
       mbar_init(&full[s], 1);
@@ -168,7 +167,7 @@ __global__ void __launch_bounds__(StreamCfg<LOGN, Tin>::THREADS, 1) k_rows_strea
     return;
   }
 
-  if (has_signs) {
+  if constexpr (SIGNS) {
     sl.store(sgn, a.pre_signs, threadIdx.x);
     asm volatile("bar.sync %0, %1;" ::"r"(C::BAR_CONSUMERS), "r"(C::NCW * 32) : "memory");
   }
@@ -215,7 +214,7 @@ __global__ void __launch_bounds__(StreamCfg<LOGN, Tin>::THREADS, 1) k_rows_strea
         bf16x2_to_f32(v.x, x[4 * j], x[4 * j + 1]);
         bf16x2_to_f32(v.y, x[4 * j + 2], x[4 * j + 3]);
       }
-      if (has_signs) {  // xor of the sign bit runs on the integer pipe, not the FP32 pipe
+      if constexpr (SIGNS) {  // xor of the sign bit runs on the integer pipe, not the FP32 pipe
         const uint4 sv = reinterpret_cast<const uint4*>(sgn)[i0 >> 2];
         x[4 * j] = __uint_as_float(__float_as_uint(x[4 * j]) ^ sv.x);
         x[4 * j + 1] = __uint_as_float(__float_as_uint(x[4 * j + 1]) ^ sv.y);
@@ -244,11 +243,11 @@ __global__ void __launch_bounds__(StreamCfg<LOGN, Tin>::THREADS, 1) k_rows_strea
   }
 }
 
-template <int LOGN, typename Tin, typename Tout, int EPI, int BITS>
-cudaError_t launch_stream(const RowArgs& a, cudaStream_t st) {
+template <int LOGN, typename Tin, typename Tout, int EPI, int BITS, bool SIGNS>
+cudaError_t launch_stream_k(const RowArgs& a, cudaStream_t st) {
   using C = StreamCfg<LOGN, Tin>;
   static std::atomic<unsigned long long> done{0};
-  auto kern = k_rows_stream<LOGN, Tin, Tout, EPI, BITS>;
+  auto kern = k_rows_stream<LOGN, Tin, Tout, EPI, BITS, SIGNS>;
   cudaError_t e = set_smem_attr(kern, C::SMEM, done);
   if (e != cudaSuccess) return e;
   int dev = 0, sms = 0;
@@ -257,6 +256,13 @@ cudaError_t launch_stream(const RowArgs& a, cudaStream_t st) {
   const int64_t grid = a.rows < sms ? a.rows : sms;
   kern<<<dim3(unsigned(grid)), C::THREADS, C::SMEM, st>>>(a);
   return cudaGetLastError();
+}
+
+// The sign flip is compiled in or out, so the row loop carries no branch on it.
+template <int LOGN, typename Tin, typename Tout, int EPI, int BITS>
+cudaError_t launch_stream(const RowArgs& a, cudaStream_t st) {
+  return a.pre_signs != nullptr ? launch_stream_k<LOGN, Tin, Tout, EPI, BITS, true>(a, st)
+                                : launch_stream_k<LOGN, Tin, Tout, EPI, BITS, false>(a, st);
 }
 
 }  // namespace hit
