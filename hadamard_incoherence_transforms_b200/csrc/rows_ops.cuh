@@ -36,6 +36,28 @@ struct QConst {
   static constexpr float MAGIC = 12582912.0f + float(1 << (BITS - 1));
 };
 
+// s = RN(a / qmax) for the group scale.  qmax is 1, 3 or 7.  For a >= 2^-120
+// the quotient is formed with the same correction step as the codes (with
+// r = RN(1/qmax) a compile-time constant): q0 = RN(a r) is within one ulp of
+// a/qmax, the remainder a - qmax q0 is exact, and RN(q0 + e r) is the
+// correctly rounded quotient; smaller a (where the remainder could underflow)
+// takes the IEEE division.
+template <int BITS>
+__device__ __forceinline__ float group_scale(float a) {
+  constexpr float QMAX = QConst<BITS>::QMAX;
+  if constexpr (BITS == 2) {
+    return a;  // qmax = 1
+  } else {
+    constexpr float R = 1.0f / QMAX;  // RN(1/qmax): 1/3 and 1/7 rounded once at compile time
+    if (a >= 0x1p-120f) {
+      const float q0 = a * R;
+      const float e = fmaf(-QMAX, q0, a);
+      return fmaf(e, R, q0);
+    }
+    return __fdiv_rn(a, QMAX);
+  }
+}
+
 // Codes of 8 elements of one group with scale s and r = RN(1/s).  An all-zero
 // group passes r = 0 (and s = 1): every quotient is then 0 and the code is
 // the offset 2^(bits-1).
@@ -115,7 +137,7 @@ __device__ __forceinline__ void quant_rowB_next(float (&x)[Geom<LOGN>::E], const
   for (int cc = 0; cc < NCH; ++cc) {
     const int e0 = E * tau + 32 * cc;
     if (cc == 0 || (e0 & ((1 << lg) - 1)) == 0) {  // first chunk of a group: its scale
-      s = __fdiv_rn(mx[cc], QMAX);
+      s = group_scale<BITS>(mx[cc]);
       if ((e0 & ((1 << lg) - 1)) == 0) a.scales[row * spr + (e0 >> lg)] = FOLD ? s * a.norm : s;
       k = s < 0x1p-100f ? 0x1p100f : (s > 0x1p100f ? 0x1p-100f : 1.0f);
       ss = s * k;

@@ -10,6 +10,10 @@
 // stages, releases the slot to the producer and runs the epilogue (store or
 // quantize + pack) from registers.  Rows in flight per SM = slots being
 // filled, so the HBM pipe stays busy while other rows are being computed.
+// Each row is copied as four quarter-row copies with a barrier each, and the
+// first wave is issued quarter by quarter: a team runs the layout-A stages
+// that stay inside a quarter (register bits 0..4) as soon as that quarter has
+// landed, so the first round of rows does not wait for whole rows.
 // Every mbarrier wait is bounded; a wait that gives up bumps a device
 // counter and the warp stops.
 #pragma once
@@ -48,13 +52,17 @@ struct StreamCfg {
   static constexpr uint32_t SIGNS = uint32_t(G::N) * 4;        // sign-bit mask per column
   static constexpr uint32_t SMEM_MAX = 232448;                 // opt-in limit per CTA on sm_100
   static constexpr int S = int((SMEM_MAX - 1024 - SIGNS) / SLOT);  // ring depth
+  static constexpr int NQ = 4;                                 // quarter copies per row
+  static constexpr uint32_t QROW = ROW / NQ;
   static constexpr size_t SMEM = 1024 + SIGNS + size_t(S) * SLOT;
   static constexpr int THREADS = (NCW + 1) * 32;
   static constexpr int BAR_CONSUMERS = 15;                     // named barrier of all consumer warps
   static_assert(TEAMS >= 1 && S + 1 >= TEAMS, "ring too shallow for the ticket protocol");
   static_assert(TEAMS + 1 < BAR_CONSUMERS, "named barrier ids");
   static_assert(S <= 32, "the ramp issues one ring slot per producer lane");
-  static_assert(2 * S * 8 + 8 + 4 * TEAMS <= 1024, "barriers and tickets must fit in the first kilobyte");
+  static_assert((NQ + 1) * S * 8 + 8 + 4 * TEAMS <= 1024, "barriers and tickets must fit in the first kilobyte");
+  static_assert(QROW % 16 == 0, "quarter copies are whole 16-byte units");
+  static_assert(G::E == 128, "quarters are the 32-register blocks of layout A");
 };
 
 template <int LOGN, typename Tin>
@@ -105,8 +113,8 @@ __global__ void __launch_bounds__(StreamCfg<LOGN, Tin>::THREADS, 1) k_rows_strea
   using G = Geom<LOGN>;
   using C = StreamCfg<LOGN, Tin>;
   extern __shared__ __align__(1024) uint8_t smem[];
-  uint64_t* full = reinterpret_cast<uint64_t*>(smem);
-  uint64_t* empty = full + C::S;
+  uint64_t* full = reinterpret_cast<uint64_t*>(smem);  // [S][NQ], one per quarter copy
+  uint64_t* empty = full + C::S * C::NQ;
   int* ticket = reinterpret_cast<int*>(empty + C::S);
   volatile int* abort = ticket + 1;
   int* team_ticket = ticket + 2;
@@ -117,7 +125,7 @@ __global__ void __launch_bounds__(StreamCfg<LOGN, Tin>::THREADS, 1) k_rows_strea
   if (SIGNS && warp < C::NCW) sl.load(a.pre_signs, threadIdx.x);
   if (threadIdx.x == 0) {
     for (int s = 0; s < C::S; ++s) {
-      mbar_init(&full[s], 1);
+      for (int q = 0; q < C::NQ; ++q) mbar_init(&full[s * C::NQ + q], 1);
       mbar_init(&empty[s], C::WPR);
     }
     ticket[0] = 0;
@@ -130,21 +138,30 @@ __global__ void __launch_bounds__(StreamCfg<LOGN, Tin>::THREADS, 1) k_rows_strea
 
   if (warp == C::NCW) {  // producer
     const uint8_t* src = static_cast<const uint8_t*>(a.x);
-    auto issue = [&](int64_t k) {
+    auto issue_q = [&](int64_t k, int q) {
       const int s = int(k % C::S);
       const int64_t row = blockIdx.x + k * grid;
-      mbar_expect_tx(&full[s], C::ROW);
-      bulk_g2s(slots + size_t(s) * C::SLOT, src + row * a.ldx * int64_t(sizeof(Tin)), C::ROW, &full[s]);
+      mbar_expect_tx(&full[s * C::NQ + q], C::QROW);
+      bulk_g2s(slots + size_t(s) * C::SLOT + size_t(q) * C::QROW,
+               src + row * a.ldx * int64_t(sizeof(Tin)) + size_t(q) * C::QROW, C::QROW, &full[s * C::NQ + q]);
     };
-    // Ramp: one row per team from parallel lanes, the rest of the ring once
-    // the first row has landed (a smaller first wave arrives sooner).
+    auto issue = [&](int64_t k) {
+#pragma unroll
+      for (int q = 0; q < C::NQ; ++q) issue_q(k, q);
+    };
+    // Ramp: one row per team from parallel lanes, quarter by quarter (all
+    // first quarters, then all second quarters, ...), and the rest of the
+    // ring once the first row has landed (a smaller first wave arrives sooner).
     const int64_t wave1 = nrows < C::TEAMS ? nrows : C::TEAMS;
     const int64_t wave2 = nrows < C::S ? nrows : C::S;
-    if (lane < wave1) issue(lane);
-    __syncwarp();
+#pragma unroll
+    for (int q = 0; q < C::NQ; ++q) {
+      if (lane < wave1) issue_q(lane, q);
+      __syncwarp();
+    }
     bool ok = true;
     if (wave2 > wave1) {
-      if (lane == 0) ok = mbar_wait(&full[0], 0u);
+      if (lane == 0) ok = mbar_wait(&full[C::NQ - 1], 0u);
       ok = __shfl_sync(0xffffffffu, ok, 0);
       if (ok && lane >= wave1 && lane < wave2) issue(lane);
       __syncwarp();
@@ -162,7 +179,8 @@ __global__ void __launch_bounds__(StreamCfg<LOGN, Tin>::THREADS, 1) k_rows_strea
       }
       // Do not leave while a copy into this CTA's shared memory is in flight.
       for (int64_t k = issued > C::S ? issued - C::S : 0; k < issued; ++k)
-        if (!mbar_wait(&full[k % C::S], uint32_t(k / C::S) & 1u)) atomicAdd(&g_wait_timeouts, 1u);
+        for (int q = 0; q < C::NQ; ++q)
+          if (!mbar_wait(&full[(k % C::S) * C::NQ + q], uint32_t(k / C::S) & 1u)) atomicAdd(&g_wait_timeouts, 1u);
     }
     return;
   }
@@ -188,41 +206,55 @@ __global__ void __launch_bounds__(StreamCfg<LOGN, Tin>::THREADS, 1) k_rows_strea
     }
     if (k >= nrows) break;
     const int s = int(k % C::S);
-    if (!mbar_wait(&full[s], uint32_t(k / C::S) & 1u)) {
-      if (lane == 0) atomicAdd(&g_wait_timeouts, 1u);
-      // A one-warp team stops here.  A two-warp team finishes the row (its
-      // partner is at the same team barriers) and both warps stop at the next
-      // ticket; the row's output is then undefined and the counter says so.
-      if constexpr (C::WPR == 1) return;
-      *abort = 1;
-    }
     const int64_t row = blockIdx.x + k * grid;
     uint8_t* slot = slots + size_t(s) * C::SLOT;
     float x[G::E];
-    // layout A straight from the copied row (linear layout)
+    // Layout A straight from the copied row (linear layout), one quarter at a
+    // time: quarter q holds vectors j = 8q .. 8q+7, i.e. registers 32q .. 32q+31,
+    // and register bits 0..4 stay inside a quarter.
+    bool stop = false;
 #pragma unroll
-    for (int j = 0; j < G::NV; ++j) {
-      const int i0 = 4 * (tau + G::T * j);
-      if constexpr (std::is_same<Tin, float>::value) {
-        const float4 v = reinterpret_cast<const float4*>(slot)[i0 >> 2];
-        x[4 * j] = v.x;
-        x[4 * j + 1] = v.y;
-        x[4 * j + 2] = v.z;
-        x[4 * j + 3] = v.w;
-      } else {
-        const uint2 v = reinterpret_cast<const uint2*>(slot)[i0 >> 2];
-        bf16x2_to_f32(v.x, x[4 * j], x[4 * j + 1]);
-        bf16x2_to_f32(v.y, x[4 * j + 2], x[4 * j + 3]);
+    for (int q = 0; q < C::NQ; ++q) {
+      if (!mbar_wait(&full[s * C::NQ + q], uint32_t(k / C::S) & 1u)) {
+        if (lane == 0) atomicAdd(&g_wait_timeouts, 1u);
+        // A one-warp team stops.  A two-warp team finishes the row (its
+        // partner is at the same team barriers) and both warps stop at the
+        // next ticket; the row's output is then undefined and the counter
+        // says so.
+        if constexpr (C::WPR == 1) stop = true;
+        else *abort = 1;
       }
-      if constexpr (SIGNS) {  // xor of the sign bit runs on the integer pipe, not the FP32 pipe
-        const uint4 sv = reinterpret_cast<const uint4*>(sgn)[i0 >> 2];
-        x[4 * j] = __uint_as_float(__float_as_uint(x[4 * j]) ^ sv.x);
-        x[4 * j + 1] = __uint_as_float(__float_as_uint(x[4 * j + 1]) ^ sv.y);
-        x[4 * j + 2] = __uint_as_float(__float_as_uint(x[4 * j + 2]) ^ sv.z);
-        x[4 * j + 3] = __uint_as_float(__float_as_uint(x[4 * j + 3]) ^ sv.w);
+      if constexpr (C::WPR == 1) {
+        if (stop) break;
       }
+#pragma unroll
+      for (int j = 8 * q; j < 8 * q + 8; ++j) {
+        const int i0 = 4 * (tau + G::T * j);
+        if constexpr (std::is_same<Tin, float>::value) {
+          const float4 v = reinterpret_cast<const float4*>(slot)[i0 >> 2];
+          x[4 * j] = v.x;
+          x[4 * j + 1] = v.y;
+          x[4 * j + 2] = v.z;
+          x[4 * j + 3] = v.w;
+        } else {
+          const uint2 v = reinterpret_cast<const uint2*>(slot)[i0 >> 2];
+          bf16x2_to_f32(v.x, x[4 * j], x[4 * j + 1]);
+          bf16x2_to_f32(v.y, x[4 * j + 2], x[4 * j + 3]);
+        }
+        if constexpr (SIGNS) {  // xor of the sign bit runs on the integer pipe, not the FP32 pipe
+          const uint4 sv = reinterpret_cast<const uint4*>(sgn)[i0 >> 2];
+          x[4 * j] = __uint_as_float(__float_as_uint(x[4 * j]) ^ sv.x);
+          x[4 * j + 1] = __uint_as_float(__float_as_uint(x[4 * j + 1]) ^ sv.y);
+          x[4 * j + 2] = __uint_as_float(__float_as_uint(x[4 * j + 2]) ^ sv.z);
+          x[4 * j + 3] = __uint_as_float(__float_as_uint(x[4 * j + 3]) ^ sv.w);
+        }
+      }
+      reg_stages<32, 0, 5>(*reinterpret_cast<float(*)[32]>(x + 32 * q));
     }
-    reg_stages<G::E, 0, G::LOGE>(x);
+    if constexpr (C::WPR == 1) {
+      if (stop) return;
+    }
+    reg_stages<G::E, 5, G::LOGE>(x);
     stream_team_sync<LOGN, Tin>(team);  // every thread has read its layout-A data
     float4* buf = reinterpret_cast<float4*>(slot);
     smem_put_A<LOGN>(buf, x, tau);
