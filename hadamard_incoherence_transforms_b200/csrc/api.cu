@@ -82,8 +82,10 @@ int run_cols(const void* src, int dt_src, int64_t ld_src, void* dst, int dt_dst,
   const int k = ilog2(m);
   const bool vec_ok = ld_src % 4 == 0 && ld_dst % 4 == 0 && aligned(src, 4 * esize(dt_src)) &&
                       aligned(dst, 4 * esize(dt_dst));
-  // One pass with clusters over 16-column strips.
-  if (k >= 10 && k <= 13 && cols % 16 == 0 && vec_ok) {
+  // One pass with clusters over 16-column strips (its staging copies are 16-byte
+  // asynchronous copies, so the source rows must start on 16-byte boundaries).
+  const bool src16 = aligned(src, 16) && (static_cast<size_t>(ld_src) * esize(dt_src)) % 16 == 0;
+  if (k >= 10 && k <= 13 && cols % 16 == 0 && vec_ok && src16) {
     hit::ColArgs a;
     a.x = src;
     a.y = dst;

@@ -236,107 +236,159 @@ cudaError_t launch_cols_full(int logm, int dt_in, int dt_out, const ColArgs& a, 
 // combined through distributed shared memory: each thread reads the CL
 // vectors of one (row, quad) position from the cluster's CTAs, runs the
 // remaining log2(CL) stages and writes the CL output rows.
+//
+// The clusters are persistent: cluster i takes strips i, i + clusters, ...,
+// and while it transforms and stores one strip its rows of the next strip
+// are already streaming into a staging buffer with 16-byte asynchronous
+// copies (cp.async), so the loads of one strip overlap the arithmetic,
+// exchange and stores of the previous one.
 // ---------------------------------------------------------------------------
-// Strip width 16 columns (4 quads): whole 32-byte sectors for bf16 rows, 64 KB
-// of shared memory and 128 threads per CTA, so three CTAs share an SM and
-// their load, exchange and store phases overlap.
 constexpr int kQuads = 4;
 constexpr int kClusterThreads = kQuads * 32;
 // 16-byte chunk of (row, quad); bit 2 is xor-ed with row bit 5 so that rows
 // 32 apart (the phase-2 pattern) fall in different bank groups.
 __device__ __forceinline__ int cs_idx(int row, int q) { return (row * kQuads + q) ^ (((row >> 5) & 1) << 2); }
 
+__device__ __forceinline__ void cp_async16(void* smem, const void* gmem) {
+  asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(smem_u32(smem)), "l"(gmem) : "memory");
+}
+__device__ __forceinline__ void cp_async_commit() { asm volatile("cp.async.commit_group;" ::: "memory"); }
+__device__ __forceinline__ void cp_async_wait_all() { asm volatile("cp.async.wait_group 0;" ::: "memory"); }
+
+template <typename Tin>
+struct ClusterSmem {
+  static constexpr int SROW = 4 * kQuads * int(sizeof(Tin));  // staged bytes per row of a strip
+  static constexpr size_t WORK = size_t(1024) * kQuads * sizeof(float4);
+  static constexpr size_t SMEM = WORK + size_t(1024) * SROW;
+};
+
 template <int CL, typename Tin, typename Tout>
 __global__ void __launch_bounds__(kClusterThreads) k_cols_cluster(const ColArgs a) {
-  extern __shared__ float4 cs_smem[];  // [1024 rows][kQuads quads]
+  using SM = ClusterSmem<Tin>;
+  extern __shared__ float4 cs_smem[];  // [1024 rows][kQuads quads] fp32, then the staging rows
+  uint8_t* stage = reinterpret_cast<uint8_t*>(cs_smem) + SM::WORK;
   namespace cg = cooperative_groups;
   cg::cluster_group cluster = cg::this_cluster();
   const int crank = static_cast<int>(cluster.block_rank());
-  const int64_t col0 = (int64_t(blockIdx.x) / CL) * (4 * kQuads);
+  const int64_t clusters = gridDim.x / CL;
+  const int64_t strips = a.cols / (4 * kQuads);
   const int tid = threadIdx.x;
   const int q = tid % kQuads;  // column quad within the strip
   const int tr = tid / kQuads;  // 0..31
   const int64_t row_base = int64_t(crank) * 1024;
-  float x[128];
-  // phase 1: rows tr + 32 k of this CTA's block
-  const Tin* src = static_cast<const Tin*>(a.x) + col0 + 4 * q;
-#pragma unroll
-  for (int k = 0; k < 32; ++k) {
-    const int64_t r = row_base + tr + 32 * k;
-    float v0, v1, v2, v3;
-    if constexpr (std::is_same<Tin, float>::value) {
-      const float4 v = __ldcs(reinterpret_cast<const float4*>(src + r * a.ldx));
-      v0 = v.x; v1 = v.y; v2 = v.z; v3 = v.w;
-    } else {
-      const uint2 v = __ldcs(reinterpret_cast<const uint2*>(src + r * a.ldx));
-      bf16x2_to_f32(v.x, v0, v1);
-      bf16x2_to_f32(v.y, v2, v3);
+  constexpr int CPR = SM::SROW / 16;  // 16-byte copies per staged row
+  auto prefetch = [&](int64_t strip) {
+    const uint8_t* src = static_cast<const uint8_t*>(a.x) + (row_base * a.ldx + strip * 4 * kQuads) * int64_t(sizeof(Tin));
+    const int64_t pitch = a.ldx * int64_t(sizeof(Tin));
+#pragma unroll 4
+    for (int i = tid; i < 1024 * CPR; i += kClusterThreads) {
+      const int r = i / CPR, c = i - r * CPR;
+      cp_async16(stage + r * SM::SROW + 16 * c, src + r * pitch + 16 * c);
     }
-    if (a.pre_signs != nullptr && a.pre_signs[r] < 0) {
-      v0 = -v0; v1 = -v1; v2 = -v2; v3 = -v3;
-    }
-    x[4 * k] = v0; x[4 * k + 1] = v1; x[4 * k + 2] = v2; x[4 * k + 3] = v3;
-  }
-  reg_stages<128, 2, 7>(x);  // row bits 5..9
-#pragma unroll
-  for (int k = 0; k < 32; ++k)
-    cs_smem[cs_idx(tr + 32 * k, q)] = make_float4(x[4 * k], x[4 * k + 1], x[4 * k + 2], x[4 * k + 3]);
-  __syncthreads();
-  // phase 2: rows 32 tr + r
-#pragma unroll
-  for (int r = 0; r < 32; ++r) {
-    const float4 v = cs_smem[cs_idx(32 * tr + r, q)];
-    x[4 * r] = v.x; x[4 * r + 1] = v.y; x[4 * r + 2] = v.z; x[4 * r + 3] = v.w;
-  }
-  reg_stages<128, 2, 7>(x);  // row bits 0..4
-  __syncthreads();           // every phase-2 read is done before the writes
-#pragma unroll
-  for (int r = 0; r < 32; ++r)
-    cs_smem[cs_idx(32 * tr + r, q)] = make_float4(x[4 * r], x[4 * r + 1], x[4 * r + 2], x[4 * r + 3]);
-  cluster.sync();  // all blocks of the strip are in shared memory
-  // phase 3: this CTA combines rows (c', row_low) for row_low in its share
-  Tout* dst = static_cast<Tout*>(a.y) + col0 + 4 * q;
+    cp_async_commit();
+  };
+
+  int64_t strip = blockIdx.x / CL;
+  if (strip < strips) prefetch(strip);
+  // Every strip of this CTA uses the same rows, so each thread's signs become
+  // two bit masks once: bit k of pre_m is the sign of phase-1 row tr + 32 k,
+  // bit 4 u + c of post_m the sign of phase-3 row 1024 c + row_low(u).
   constexpr int SHARE = 1024 / CL;
-#pragma unroll 1
-  for (int u = 0; u < SHARE / 32; ++u) {
-    const int row_low = crank * SHARE + tr + 32 * u;
-    float v[4 * CL];
+  uint32_t pre_m = 0, post_m = 0;
+  if (a.pre_signs != nullptr) {
 #pragma unroll
-    for (int c = 0; c < CL; ++c) {
-      const float4* rem = cluster.map_shared_rank(cs_smem, c);
-      const float4 w = rem[cs_idx(row_low, q)];
-      v[4 * c] = w.x; v[4 * c + 1] = w.y; v[4 * c + 2] = w.z; v[4 * c + 3] = w.w;
-    }
-    if constexpr (CL > 1) reg_stages<4 * CL, 2, 2 + (CL == 2 ? 1 : (CL == 4 ? 2 : 3))>(v);
-#pragma unroll
-    for (int c = 0; c < CL; ++c) {
-      const int64_t r = int64_t(c) * 1024 + row_low;
-      float o0 = v[4 * c] * a.norm, o1 = v[4 * c + 1] * a.norm, o2 = v[4 * c + 2] * a.norm, o3 = v[4 * c + 3] * a.norm;
-      if (a.post_signs != nullptr && a.post_signs[r] < 0) {
-        o0 = -o0; o1 = -o1; o2 = -o2; o3 = -o3;
-      }
-      if constexpr (std::is_same<Tout, float>::value) {
-        __stcs(reinterpret_cast<float4*>(dst + r * a.ldy), make_float4(o0, o1, o2, o3));
-      } else {
-        __stcs(reinterpret_cast<uint2*>(dst + r * a.ldy), make_uint2(f32_to_bf16x2(o0, o1), f32_to_bf16x2(o2, o3)));
-      }
-    }
+    for (int k = 0; k < 32; ++k) pre_m |= uint32_t(a.pre_signs[row_base + tr + 32 * k] < 0) << k;
   }
-  cluster.sync();  // no CTA leaves while others still read its shared memory
+  if (a.post_signs != nullptr) {
+#pragma unroll
+    for (int u = 0; u < SHARE / 32; ++u)
+#pragma unroll
+      for (int c = 0; c < CL; ++c)
+        post_m |= uint32_t(a.post_signs[int64_t(c) * 1024 + crank * SHARE + tr + 32 * u] < 0) << (u * CL + c);
+  }
+  for (; strip < strips; strip += clusters) {
+    cp_async_wait_all();
+    __syncthreads();  // every thread's copies of this strip have landed
+    float x[128];
+    // phase 1: rows tr + 32 k of this CTA's block, from the staging rows
+#pragma unroll
+    for (int k = 0; k < 32; ++k) {
+      const int r = tr + 32 * k;
+      float v0, v1, v2, v3;
+      if constexpr (std::is_same<Tin, float>::value) {
+        const float4 v = *reinterpret_cast<const float4*>(stage + r * SM::SROW + 16 * q);
+        v0 = v.x; v1 = v.y; v2 = v.z; v3 = v.w;
+      } else {
+        const uint2 v = *reinterpret_cast<const uint2*>(stage + r * SM::SROW + 8 * q);
+        bf16x2_to_f32(v.x, v0, v1);
+        bf16x2_to_f32(v.y, v2, v3);
+      }
+      const uint32_t sb = (pre_m >> k) << 31;
+      x[4 * k] = __uint_as_float(__float_as_uint(v0) ^ sb);
+      x[4 * k + 1] = __uint_as_float(__float_as_uint(v1) ^ sb);
+      x[4 * k + 2] = __uint_as_float(__float_as_uint(v2) ^ sb);
+      x[4 * k + 3] = __uint_as_float(__float_as_uint(v3) ^ sb);
+    }
+    __syncthreads();  // the staging rows are free: start streaming the next strip
+    if (strip + clusters < strips) prefetch(strip + clusters);
+    reg_stages<128, 2, 7>(x);  // row bits 5..9
+#pragma unroll
+    for (int k = 0; k < 32; ++k)
+      cs_smem[cs_idx(tr + 32 * k, q)] = make_float4(x[4 * k], x[4 * k + 1], x[4 * k + 2], x[4 * k + 3]);
+    __syncthreads();
+    // phase 2: rows 32 tr + r
+#pragma unroll
+    for (int r = 0; r < 32; ++r) {
+      const float4 v = cs_smem[cs_idx(32 * tr + r, q)];
+      x[4 * r] = v.x; x[4 * r + 1] = v.y; x[4 * r + 2] = v.z; x[4 * r + 3] = v.w;
+    }
+    reg_stages<128, 2, 7>(x);  // row bits 0..4
+    __syncthreads();           // every phase-2 read is done before the writes
+#pragma unroll
+    for (int r = 0; r < 32; ++r)
+      cs_smem[cs_idx(32 * tr + r, q)] = make_float4(x[4 * r], x[4 * r + 1], x[4 * r + 2], x[4 * r + 3]);
+    cluster.sync();  // all blocks of the strip are in shared memory
+    // phase 3: this CTA combines rows (c', row_low) for row_low in its share
+    Tout* dst = static_cast<Tout*>(a.y) + strip * 4 * kQuads + 4 * q;
+#pragma unroll
+    for (int u = 0; u < SHARE / 32; ++u) {
+      const int row_low = crank * SHARE + tr + 32 * u;
+      float v[4 * CL];
+#pragma unroll
+      for (int c = 0; c < CL; ++c) {
+        const float4* rem = cluster.map_shared_rank(cs_smem, c);
+        const float4 w = rem[cs_idx(row_low, q)];
+        v[4 * c] = w.x; v[4 * c + 1] = w.y; v[4 * c + 2] = w.z; v[4 * c + 3] = w.w;
+      }
+      if constexpr (CL > 1) reg_stages<4 * CL, 2, 2 + (CL == 2 ? 1 : (CL == 4 ? 2 : 3))>(v);
+#pragma unroll
+      for (int c = 0; c < CL; ++c) {
+        const int64_t r = int64_t(c) * 1024 + row_low;
+        const float nrm = __uint_as_float(__float_as_uint(a.norm) ^ (((post_m >> (u * CL + c)) & 1u) << 31));
+        const float o0 = v[4 * c] * nrm, o1 = v[4 * c + 1] * nrm, o2 = v[4 * c + 2] * nrm, o3 = v[4 * c + 3] * nrm;
+        if constexpr (std::is_same<Tout, float>::value) {
+          __stcs(reinterpret_cast<float4*>(dst + r * a.ldy), make_float4(o0, o1, o2, o3));
+        } else {
+          __stcs(reinterpret_cast<uint2*>(dst + r * a.ldy), make_uint2(f32_to_bf16x2(o0, o1), f32_to_bf16x2(o2, o3)));
+        }
+      }
+    }
+    cluster.sync();  // no CTA rewrites its block while others still read it
+  }
+  cp_async_wait_all();  // nothing in flight into this CTA's shared memory at exit
 }
 
 template <int CL, typename Tin, typename Tout>
 static cudaError_t launch_cluster_t(const ColArgs& a, cudaStream_t st) {
+  using SM = ClusterSmem<Tin>;
   auto kern = k_cols_cluster<CL, Tin, Tout>;
-  constexpr size_t smem = size_t(1024) * kQuads * sizeof(float4);
   static std::atomic<unsigned long long> done{0};
-  cudaError_t e = set_smem_attr(kern, smem, done);
+  cudaError_t e = set_smem_attr(kern, SM::SMEM, done);
   if (e != cudaSuccess) return e;
   const int64_t strips = a.cols / (4 * kQuads);
   cudaLaunchConfig_t cfg = {};
-  cfg.gridDim = dim3(static_cast<unsigned>(strips * CL));
   cfg.blockDim = dim3(kClusterThreads);
-  cfg.dynamicSmemBytes = smem;
+  cfg.dynamicSmemBytes = SM::SMEM;
   cfg.stream = st;
   cudaLaunchAttribute attr[1];
   attr[0].id = cudaLaunchAttributeClusterDimension;
@@ -345,6 +397,20 @@ static cudaError_t launch_cluster_t(const ColArgs& a, cudaStream_t st) {
   attr[0].val.clusterDim.z = 1;
   cfg.attrs = attr;
   cfg.numAttrs = 1;
+  // Persistent clusters: as many as can be resident at once (queried once per
+  // device), never more than there are strips.
+  static std::atomic<int> resident[64];
+  int dev = 0;
+  if ((e = cudaGetDevice(&dev)) != cudaSuccess) return e;
+  int nres = dev < 64 ? resident[dev].load() : 0;
+  if (nres <= 0) {
+    cfg.gridDim = dim3(static_cast<unsigned>(CL));
+    if ((e = cudaOccupancyMaxActiveClusters(&nres, kern, &cfg)) != cudaSuccess) return e;
+    if (nres <= 0) nres = 1;
+    if (dev < 64) resident[dev].store(nres);
+  }
+  const int64_t clusters = strips < nres ? strips : nres;
+  cfg.gridDim = dim3(static_cast<unsigned>(clusters * CL));
   e = cudaLaunchKernelEx(&cfg, kern, a);
   if (e != cudaSuccess) return e;
   return cudaGetLastError();
