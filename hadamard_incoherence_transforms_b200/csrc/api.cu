@@ -233,7 +233,7 @@ static bool plan_pass(const int* order, int cnt, const int32_t* radices, const i
     }
     const int64_t pnl = P * NL;
     const int64_t pitch = (pnl % 2 == 0) ? pnl + 1 : pnl;
-    for (int log_nb = 8; log_nb >= 0; --log_nb) {
+    for (int log_nb = 10; log_nb >= 0; --log_nb) {
       const int64_t nb = int64_t(1) << log_nb;
       const size_t bytes = static_cast<size_t>(blk + nb * pitch) * sizeof(float);
       if (bytes > budget || nb * pnl > 32768) continue;
@@ -272,6 +272,7 @@ static bool plan_pass(const int* order, int cnt, const int32_t* radices, const i
     st.bp = (st.b + 3) / 4 * 4;
     st.ls = static_cast<int>(S[t] / S_in);
     st.div_ls = hit::make_fastdiv(static_cast<uint32_t>(st.ls));
+    st.div_bp = hit::make_fastdiv(static_cast<uint32_t>(st.bp));
     st.sofs = ofs;
     st.shared_block = (n_groups[t] == 1 && len / radices[t] != 1) ? 1 : 0;
     st.transpose = transpose ? 1 : 0;

@@ -31,12 +31,127 @@ __device__ __forceinline__ uint32_t fdiv(uint32_t n, const FastDiv& f) {
   return (__umulhi(n, f.mul) + n) >> f.shr;
 }
 
+// Offset, inside a tile row, of the first position of local group g of a
+// stage with radix b (the group's positions follow at stride ls << log_nl).
+__device__ __forceinline__ int group_offset(int g, int b, const BflyStage& st, int log_nl, int nlm) {
+  const int mp = g >> log_nl, l = g & nlm;
+  const int mh = int(fdiv(uint32_t(mp), st.div_ls)), ml = mp - mh * st.ls;
+  return ((mh * b * st.ls + ml) << log_nl) + l;
+}
+
+// A stage of fixed radix B: a thread takes R rows of one group (rows rq,
+// rq + NB/R, ...) and streams the B inputs: per input k it loads its R input
+// values and the block's row k (the coefficients of all B outputs, one
+// 16-byte broadcast per four outputs) and updates R x B accumulators with
+// packed FMAs, so every coefficient loaded feeds R rows.  Items own disjoint
+// (row, position) sets and read all their inputs before writing, so the stage
+// runs in place.
+template <int B, int R>
+__device__ __forceinline__ void stage_fixed(float* tile, const float* sblk, const BflyStage& st, int groups,
+                                            int log_nb, int pitch, int log_nl, int nlm) {
+  constexpr int BP = (B + 3) / 4 * 4;
+  constexpr int LR = R == 4 ? 2 : (R == 2 ? 1 : 0);
+  const int log_nbr = log_nb - LR;
+  const int nbr = 1 << log_nbr;
+  const int items = groups << log_nbr;
+  const int step = st.ls << log_nl;
+  for (int it = threadIdx.x; it < items; it += blockDim.x) {
+    const int rq = it & (nbr - 1);
+    const int g = it >> log_nbr;
+    const int off = group_offset(g, B, st, log_nl, nlm);
+    int rows[R];  // tile offsets of the item's rows
+#pragma unroll
+    for (int r = 0; r < R; ++r) rows[r] = (rq + r * nbr) * pitch + off;
+    const float4* blk = reinterpret_cast<const float4*>(sblk + st.sofs + (st.shared_block ? 0 : g * B * BP));
+    float acc[R][BP];
+#pragma unroll
+    for (int r = 0; r < R; ++r)
+#pragma unroll
+      for (int j = 0; j < BP; ++j) acc[r][j] = 0.0f;
+#pragma unroll
+    for (int k = 0; k < B; ++k) {
+      float xk[R];
+#pragma unroll
+      for (int r = 0; r < R; ++r) xk[r] = tile[rows[r] + k * step];
+#pragma unroll
+      for (int j4 = 0; j4 < BP / 4; ++j4) {
+        const float4 w = blk[(k * BP >> 2) + j4];
+#pragma unroll
+        for (int r = 0; r < R; ++r) {
+          fma_x2(w.x, w.y, xk[r], xk[r], acc[r][4 * j4], acc[r][4 * j4 + 1], acc[r][4 * j4], acc[r][4 * j4 + 1]);
+          fma_x2(w.z, w.w, xk[r], xk[r], acc[r][4 * j4 + 2], acc[r][4 * j4 + 3], acc[r][4 * j4 + 2],
+                 acc[r][4 * j4 + 3]);
+        }
+      }
+    }
+#pragma unroll
+    for (int r = 0; r < R; ++r)
+#pragma unroll
+      for (int j = 0; j < B; ++j) tile[rows[r] + j * step] = acc[r][j];
+  }
+}
+
+// Any radix b <= BM: one thread per (row, group) item, all b accumulators in
+// registers.
+template <int BM>
+__device__ __forceinline__ void stage_generic(float* tile, const float* sblk, const BflyStage& st, int groups,
+                                              int log_nb, int pitch, int log_nl, int nlm) {
+  const int b = st.b, bp = st.bp;
+  const int items = groups << log_nb;
+  const int nbm = (1 << log_nb) - 1;
+  const int step = st.ls << log_nl;
+  for (int it = threadIdx.x; it < items; it += blockDim.x) {
+    const int bi = it & nbm;
+    const int g = it >> log_nb;
+    float* row = tile + bi * pitch + group_offset(g, b, st, log_nl, nlm);
+    float v[BM];
+#pragma unroll
+    for (int k = 0; k < BM; ++k) v[k] = k < b ? row[k * step] : 0.0f;
+    float acc[BM];
+#pragma unroll
+    for (int j = 0; j < BM; ++j) acc[j] = 0.0f;
+    const float4* blk = reinterpret_cast<const float4*>(sblk + st.sofs + (st.shared_block ? 0 : g * b * bp));
+#pragma unroll
+    for (int k = 0; k < BM; ++k) {
+      if (k < b) {
+#pragma unroll
+        for (int j4 = 0; j4 < BM / 4; ++j4) {
+          if (4 * j4 < bp) {
+            const float4 w = blk[(k * bp >> 2) + j4];
+            fma_x2(w.x, w.y, v[k], v[k], acc[4 * j4], acc[4 * j4 + 1], acc[4 * j4], acc[4 * j4 + 1]);
+            fma_x2(w.z, w.w, v[k], v[k], acc[4 * j4 + 2], acc[4 * j4 + 3], acc[4 * j4 + 2], acc[4 * j4 + 3]);
+          }
+        }
+      }
+    }
+#pragma unroll
+    for (int j = 0; j < BM; ++j)
+      if (j < b) row[j * step] = acc[j];
+  }
+}
+
+template <int BM, int B>
+__device__ __forceinline__ bool try_fixed(float* tile, const float* sblk, const BflyStage& st, int groups, int log_nb,
+                                          int pitch, int log_nl, int nlm) {
+  // four rows per thread (two for radix 16, whose 64 accumulators would not
+  // leave room for two CTAs per SM)
+  constexpr int R = B >= 16 ? 2 : 4;
+  if constexpr (B <= BM) {
+    if (st.b == B && log_nb >= (R == 4 ? 2 : 1)) {
+      stage_fixed<B, R>(tile, sblk, st, groups, log_nb, pitch, log_nl, nlm);
+      return true;
+    }
+  }
+  return false;
+}
+
 template <int BM, typename Tin, typename Tout>
 __global__ void __launch_bounds__(256, 2) k_bfly_pass(const BflyPass p) {  // launched with 256 threads, up to two CTAs per SM
   extern __shared__ float4 bf_smem4[];
   float* sblk = reinterpret_cast<float*>(bf_smem4);  // per stage: [group][k][bp] (bp >= b, zero padded)
   float* tile = sblk + p.blk_floats;                  // [NB][pitch]
   const int tid = threadIdx.x;
+  const int warp = tid >> 5, lane = tid & 31, nwarps = blockDim.x >> 5;
   const int64_t tiles_lo = p.S_in >> p.log_nl;
   const int64_t tile_id = int64_t(blockIdx.x) % p.n_tiles;
   const int64_t split = int64_t(blockIdx.x) / p.n_tiles;
@@ -44,128 +159,126 @@ __global__ void __launch_bounds__(256, 2) k_bfly_pass(const BflyPass p) {  // la
   const int64_t lo0 = (tile_id % tiles_lo) << p.log_nl;
   const int64_t base = hi * p.P * p.S_in + lo0;  // position of (mid = 0, l = 0)
   const int PNL = p.P << p.log_nl;
-  const int nlm = p.NL - 1, nbm = p.NB - 1;
+  const int nlm = p.NL - 1;
 
   // 1. this tile's blocks -> shared memory, laid out so that for a fixed input
   //    index k the b output coefficients are contiguous: row k holds
-  //    B[j][k] (forward) or B[k][j] (transpose) for j = 0 .. b-1.
+  //    B[j][k] (forward) or B[k][j] (transpose) for j = 0 .. b-1.  One warp
+  //    per group.
   for (int s = 0; s < p.ns; ++s) {
     const BflyStage& st = p.st[s];
-    const int b = st.b, bb = b * b, bp = st.bp;
+    const int b = st.b, bp = st.bp, kjn = b * bp;
     const int groups = st.shared_block ? 1 : (p.P / b) << p.log_nl;
     float* dst = sblk + st.sofs;
-    for (int i = tid; i < groups * b * bp; i += blockDim.x) {
-      const int g = i / (b * bp), r = i - g * (b * bp);
-      const int k = r / bp, j = r - k * bp;
-      float v = 0.0f;
-      if (j < b) {
-        int64_t c = 0;
-        if (!st.shared_block) {
-          const int mp = g >> p.log_nl, l = g & nlm;
-          c = hi * (p.P / b) * p.S_in + int64_t(mp) * p.S_in + lo0 + l;
-        }
-        v = __ldg(st.blocks + c * bb + (st.transpose ? k * b + j : j * b + k));
+    for (int g = warp; g < groups; g += nwarps) {
+      const float* src_blk = st.blocks;
+      if (!st.shared_block) {
+        const int mp = g >> p.log_nl, l = g & nlm;
+        src_blk += (hi * (p.P / b) * p.S_in + int64_t(mp) * p.S_in + lo0 + l) * int64_t(b) * b;
       }
-      dst[i] = v;
+      for (int kj = lane; kj < kjn; kj += 32) {
+        const int k = int(fdiv(uint32_t(kj), st.div_bp)), j = kj - k * bp;
+        dst[g * kjn + kj] = j < b ? __ldg(src_blk + (st.transpose ? k * b + j : j * b + k)) : 0.0f;
+      }
     }
   }
 
   const Tin* src = static_cast<const Tin*>(p.x);
   Tout* out = static_cast<Tout*>(p.y);
+  // Fixed per-thread share of the tile for loads and stores.  Along rows
+  // (axis 1) a thread keeps position q and walks rows bi, bi + R0, ...;
+  // along columns (axis 0) the lanes walk consecutive columns bi (contiguous
+  // in memory) and the warps take positions.
+  const int QS = PNL < int(blockDim.x) ? PNL : int(blockDim.x);
+  const int R0 = int(blockDim.x) / QS;
+  const int qi = tid % QS, ri = tid / QS;
+  const int BS = p.NB < 32 ? p.NB : 32;
+  const int bl = tid % BS, qw0 = tid / BS, QW = int(blockDim.x) / BS;
+
   const int64_t chunk0 = split * p.chunks_per_split;
   for (int64_t ch = chunk0; ch < chunk0 + p.chunks_per_split; ++ch) {
     const int64_t o0 = ch << p.log_nb;  // first row (axis 1) / column (axis 0) of this chunk
     if (o0 >= p.outer) break;
     const int nb = int(p.outer - o0 < p.NB ? p.outer - o0 : p.NB);
     __syncthreads();  // blocks ready / previous chunk stored
-    // 2. load the tile (consecutive threads: consecutive memory),
-    //    sixteen independent loads in flight per thread before they land in shared memory
-    constexpr int U = 16;
-    const int total = PNL << p.log_nb;
-    for (int e0 = tid; e0 < total; e0 += U * blockDim.x) {
-      float val[U];
-      int dst[U];
+    // 2. load the tile
+    if (p.axis == 1) {
+      if (ri < R0) {
+        for (int q = qi; q < PNL; q += QS) {
+          const int64_t coff = base + int64_t(q >> p.log_nl) * p.S_in + (q & nlm);
+          const Tin* sp = src + (o0 + ri) * p.ldx + coff;
+          float* tp = tile + ri * p.pitch + q;
+          const int64_t sstep = int64_t(R0) * p.ldx;
+          const int tstep = R0 * p.pitch;
+          int bi = ri;
+          for (; bi + 7 * R0 < nb; bi += 8 * R0) {  // eight loads in flight
+            float v[8];
 #pragma unroll
-      for (int u = 0; u < U; ++u) {
-        const int e = e0 + u * blockDim.x;
-        dst[u] = -1;
-        val[u] = 0.0f;
-        if (e < total) {
-          int bi, q;
-          if (p.axis == 1) {
-            bi = int(fdiv(uint32_t(e), p.div_pnl));
-            q = e - bi * PNL;
-          } else {
-            bi = e & nbm;
-            q = e >> p.log_nb;
+            for (int u = 0; u < 8; ++u) {
+              v[u] = to_f32(__ldcs(sp));
+              sp += sstep;
+            }
+#pragma unroll
+            for (int u = 0; u < 8; ++u) tp[u * tstep] = v[u];
+            tp += 8 * tstep;
           }
-          if (bi < nb) {
-            const int64_t pos = base + int64_t(q >> p.log_nl) * p.S_in + (q & nlm);
-            const int64_t g = p.axis == 1 ? (o0 + bi) * p.ldx + pos : pos * p.ldx + (o0 + bi);
-            val[u] = to_f32(__ldcs(src + g));
-            dst[u] = bi * p.pitch + q;
+          for (; bi < nb; bi += R0) {
+            *tp = to_f32(__ldcs(sp));
+            sp += sstep;
+            tp += tstep;
           }
         }
       }
+    } else {
+      for (int q = qw0; q < PNL; q += QW) {
+        const int64_t r = base + int64_t(q >> p.log_nl) * p.S_in + (q & nlm);
+        const Tin* sp = src + r * p.ldx + o0;
+        int bi = bl;
+        for (; bi + 7 * BS < nb; bi += 8 * BS) {  // eight loads in flight
+          float v[8];
 #pragma unroll
-      for (int u = 0; u < U; ++u)
-        if (dst[u] >= 0) tile[dst[u]] = val[u];
+          for (int u = 0; u < 8; ++u) v[u] = to_f32(__ldcs(sp + bi + u * BS));
+#pragma unroll
+          for (int u = 0; u < 8; ++u) tile[(bi + u * BS) * p.pitch + q] = v[u];
+        }
+        for (; bi < nb; bi += BS) tile[bi * p.pitch + q] = to_f32(__ldcs(sp + bi));
+      }
     }
     __syncthreads();
     // 3. the stages, in application order
     for (int s = 0; s < p.ns; ++s) {
       const BflyStage& st = p.st[s];
-      const int b = st.b, bp = st.bp, ls = st.ls;
-      const int items = ((p.P / b) << p.log_nl) << p.log_nb;
-      for (int it = tid; it < items; it += blockDim.x) {
-        const int bi = it & nbm;
-        const int g = it >> p.log_nb;  // local group (m', l)
-        const int mp = g >> p.log_nl, l = g & nlm;
-        const int mh = int(fdiv(uint32_t(mp), st.div_ls)), ml = mp - mh * ls;
-        const int mid0 = mh * b * ls + ml;
-        float* row = tile + bi * p.pitch + l;
-        const int step = ls << p.log_nl;
-        float v[BM];
-#pragma unroll
-        for (int k = 0; k < BM; ++k) v[k] = k < b ? row[(mid0 << p.log_nl) + k * step] : 0.0f;
-        float acc[BM];
-#pragma unroll
-        for (int j = 0; j < BM; ++j) acc[j] = 0.0f;
-        const float4* blk = reinterpret_cast<const float4*>(sblk + st.sofs + (st.shared_block ? 0 : g * b * bp));
-#pragma unroll
-        for (int k = 0; k < BM; ++k) {
-          if (k < b) {
-#pragma unroll
-            for (int j4 = 0; j4 < BM / 4; ++j4) {
-              if (4 * j4 < bp) {
-                const float4 w = blk[(k * bp >> 2) + j4];
-                fma_x2(w.x, w.y, v[k], v[k], acc[4 * j4], acc[4 * j4 + 1], acc[4 * j4], acc[4 * j4 + 1]);
-                fma_x2(w.z, w.w, v[k], v[k], acc[4 * j4 + 2], acc[4 * j4 + 3], acc[4 * j4 + 2], acc[4 * j4 + 3]);
-              }
-            }
-          }
-        }
-#pragma unroll
-        for (int j = 0; j < BM; ++j)
-          if (j < b) row[(mid0 << p.log_nl) + j * step] = acc[j];
-      }
+      const int groups = (p.P / st.b) << p.log_nl;
+      if (!(try_fixed<BM, 16>(tile, sblk, st, groups, p.log_nb, p.pitch, p.log_nl, nlm) ||
+            try_fixed<BM, 8>(tile, sblk, st, groups, p.log_nb, p.pitch, p.log_nl, nlm) ||
+            try_fixed<BM, 7>(tile, sblk, st, groups, p.log_nb, p.pitch, p.log_nl, nlm) ||
+            try_fixed<BM, 4>(tile, sblk, st, groups, p.log_nb, p.pitch, p.log_nl, nlm) ||
+            try_fixed<BM, 2>(tile, sblk, st, groups, p.log_nb, p.pitch, p.log_nl, nlm)))
+        stage_generic<BM>(tile, sblk, st, groups, p.log_nb, p.pitch, p.log_nl, nlm);
       __syncthreads();
     }
     // 4. store the tile
-#pragma unroll 4
-    for (int e = tid; e < (PNL << p.log_nb); e += blockDim.x) {
-      int bi, q;
-      if (p.axis == 1) {
-        bi = int(fdiv(uint32_t(e), p.div_pnl));
-        q = e - bi * PNL;
-      } else {
-        bi = e & nbm;
-        q = e >> p.log_nb;
+    if (p.axis == 1) {
+      if (ri < R0) {
+        for (int q = qi; q < PNL; q += QS) {
+          const int64_t coff = base + int64_t(q >> p.log_nl) * p.S_in + (q & nlm);
+          Tout* dp = out + (o0 + ri) * p.ldy + coff;
+          const float* tp = tile + ri * p.pitch + q;
+          const int64_t dstep = int64_t(R0) * p.ldy;
+          const int tstep = R0 * p.pitch;
+          for (int bi = ri; bi < nb; bi += R0) {
+            __stcs(dp, from_f32<Tout>(*tp));
+            dp += dstep;
+            tp += tstep;
+          }
+        }
       }
-      if (bi >= nb) continue;
-      const int64_t pos = base + int64_t(q >> p.log_nl) * p.S_in + (q & nlm);
-      const int64_t g = p.axis == 1 ? (o0 + bi) * p.ldy + pos : pos * p.ldy + (o0 + bi);
-      __stcs(out + g, from_f32<Tout>(tile[bi * p.pitch + q]));
+    } else {
+      for (int q = qw0; q < PNL; q += QW) {
+        const int64_t r = base + int64_t(q >> p.log_nl) * p.S_in + (q & nlm);
+        Tout* dp = out + r * p.ldy + o0;
+        for (int bi = bl; bi < nb; bi += BS) __stcs(dp + bi, from_f32<Tout>(tile[bi * p.pitch + q]));
+      }
     }
   }
 }

@@ -88,6 +88,7 @@ struct BflyStage {
   int bp = 4;                     // b rounded up to a multiple of 4 (shared-memory row length)
   int ls = 1;                     // stride of this digit inside the group index mid
   FastDiv div_ls;                 // division by ls
+  FastDiv div_bp;                 // division by bp
   int sofs = 0;                   // float offset of the stage's blocks in shared memory
   int shared_block = 0;
   int transpose = 0;              // use B^T
