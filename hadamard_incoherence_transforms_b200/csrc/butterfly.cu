@@ -31,6 +31,12 @@ __device__ __forceinline__ uint32_t fdiv(uint32_t n, const FastDiv& f) {
   return (__umulhi(n, f.mul) + n) >> f.shr;
 }
 
+// One fp32 element global -> shared without passing through registers, so a
+// thread can have all of its tile loads in flight at once.
+__device__ __forceinline__ void cp_async4(float* smem, const float* gmem) {
+  asm volatile("cp.async.ca.shared.global [%0], [%1], 4;" ::"r"(smem_u32(smem)), "l"(gmem) : "memory");
+}
+
 // Offset, inside a tile row, of the first position of local group g of a
 // stage with radix b (the group's positions follow at stride ls << log_nl).
 __device__ __forceinline__ int group_offset(int g, int b, const BflyStage& st, int log_nl, int nlm) {
@@ -202,7 +208,33 @@ __global__ void __launch_bounds__(256, 2) k_bfly_pass(const BflyPass p) {  // la
     const int nb = int(p.outer - o0 < p.NB ? p.outer - o0 : p.NB);
     __syncthreads();  // blocks ready / previous chunk stored
     // 2. load the tile
-    if (p.axis == 1) {
+    if constexpr (std::is_same<Tin, float>::value) {
+      // fp32 input: every element of the tile is an asynchronous copy
+      if (p.axis == 1) {
+        if (ri < R0) {
+          for (int q = qi; q < PNL; q += QS) {
+            const int64_t coff = base + int64_t(q >> p.log_nl) * p.S_in + (q & nlm);
+            const float* sp = src + (o0 + ri) * p.ldx + coff;
+            float* tp = tile + ri * p.pitch + q;
+            const int64_t sstep = int64_t(R0) * p.ldx;
+            const int tstep = R0 * p.pitch;
+            for (int bi = ri; bi < nb; bi += R0) {
+              cp_async4(tp, sp);
+              sp += sstep;
+              tp += tstep;
+            }
+          }
+        }
+      } else {
+        for (int q = qw0; q < PNL; q += QW) {
+          const int64_t r = base + int64_t(q >> p.log_nl) * p.S_in + (q & nlm);
+          const float* sp = src + r * p.ldx + o0;
+          for (int bi = bl; bi < nb; bi += BS) cp_async4(tile + bi * p.pitch + q, sp + bi);
+        }
+      }
+      asm volatile("cp.async.commit_group;" ::: "memory");
+      asm volatile("cp.async.wait_group 0;" ::: "memory");
+    } else if (p.axis == 1) {
       if (ri < R0) {
         for (int q = qi; q < PNL; q += QS) {
           const int64_t coff = base + int64_t(q >> p.log_nl) * p.S_in + (q & nlm);
