@@ -128,6 +128,13 @@ __device__ __forceinline__ float4 ld_stream_f4(const float* p) { return __ldcs(r
 __device__ __forceinline__ uint2 ld_stream_u2(const void* p) { return __ldcs(reinterpret_cast<const uint2*>(p)); }
 __device__ __forceinline__ void st_stream_f4(float* p, float4 v) { __stcs(reinterpret_cast<float4*>(p), v); }
 __device__ __forceinline__ void st_stream_u2(void* p, uint2 v) { __stcs(reinterpret_cast<uint2*>(p), v); }
+// 32-byte streaming store (one whole sector per thread); p must be 32-byte aligned.
+__device__ __forceinline__ void st_stream_v8(void* p, uint32_t a0, uint32_t a1, uint32_t a2, uint32_t a3, uint32_t a4,
+                                             uint32_t a5, uint32_t a6, uint32_t a7) {
+  asm volatile("st.global.cs.v8.b32 [%0], {%1, %2, %3, %4, %5, %6, %7, %8};" ::"l"(p), "r"(a0), "r"(a1), "r"(a2),
+               "r"(a3), "r"(a4), "r"(a5), "r"(a6), "r"(a7)
+               : "memory");
+}
 
 // ---------------------------------------------------------------------------
 // Row-buffer swizzle for the register-layout transposes.  The buffer is

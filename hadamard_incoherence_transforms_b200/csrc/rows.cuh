@@ -175,6 +175,31 @@ __device__ __forceinline__ void store_rowB(float (&x)[Geom<LOGN>::E], Tout* __re
         if (sg[base + e] < 0) x[e] = -x[e];
     }
   }
+  // A thread's run is contiguous: with 32-byte alignment it goes out as whole
+  // 32-byte sectors, one per store.
+  const bool wide = (reinterpret_cast<uintptr_t>(dst + base) & 31) == 0;
+  if constexpr (std::is_same<Tout, float>::value && E >= 8) {
+    if (wide) {
+#pragma unroll
+      for (int m = 0; m < E / 8; ++m)
+        st_stream_v8(dst + base + 8 * m, __float_as_uint(x[8 * m]), __float_as_uint(x[8 * m + 1]),
+                     __float_as_uint(x[8 * m + 2]), __float_as_uint(x[8 * m + 3]), __float_as_uint(x[8 * m + 4]),
+                     __float_as_uint(x[8 * m + 5]), __float_as_uint(x[8 * m + 6]), __float_as_uint(x[8 * m + 7]));
+      return;
+    }
+  }
+  if constexpr (std::is_same<Tout, __nv_bfloat16>::value && E >= 16) {
+    if (wide) {
+#pragma unroll
+      for (int m = 0; m < E / 16; ++m)
+        st_stream_v8(dst + base + 16 * m, f32_to_bf16x2(x[16 * m], x[16 * m + 1]),
+                     f32_to_bf16x2(x[16 * m + 2], x[16 * m + 3]), f32_to_bf16x2(x[16 * m + 4], x[16 * m + 5]),
+                     f32_to_bf16x2(x[16 * m + 6], x[16 * m + 7]), f32_to_bf16x2(x[16 * m + 8], x[16 * m + 9]),
+                     f32_to_bf16x2(x[16 * m + 10], x[16 * m + 11]), f32_to_bf16x2(x[16 * m + 12], x[16 * m + 13]),
+                     f32_to_bf16x2(x[16 * m + 14], x[16 * m + 15]));
+      return;
+    }
+  }
   if constexpr (std::is_same<Tout, float>::value && E >= 4) {
 #pragma unroll
     for (int m = 0; m < E / 4; ++m)

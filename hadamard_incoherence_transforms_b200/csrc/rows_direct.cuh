@@ -109,6 +109,7 @@ __device__ __forceinline__ void store_rowB_next(float (&x)[Geom<LOGN>::E], Tout*
   using G = Geom<LOGN>;
   constexpr int E = G::E;
   const int base = E * tau;
+  const bool wide = (reinterpret_cast<uintptr_t>(dst + base) & 31) == 0;
 #pragma unroll
   for (int cc = 0; cc < E / 32; ++cc) {
     float* xc = x + 32 * cc;
@@ -121,10 +122,19 @@ __device__ __forceinline__ void store_rowB_next(float (&x)[Geom<LOGN>::E], Tout*
                     __ldg(reinterpret_cast<const uint32_t*>(sg + base + 32 * cc + 4 * m)));
     }
     if constexpr (std::is_same<Tout, float>::value) {
+      if (!wide) {
 #pragma unroll
-      for (int m = 0; m < 8; ++m)
-        st_stream_f4(dst + base + 32 * cc + 4 * m, make_float4(xc[4 * m], xc[4 * m + 1], xc[4 * m + 2], xc[4 * m + 3]));
-    } else {
+        for (int m = 0; m < 8; ++m)
+          st_stream_f4(dst + base + 32 * cc + 4 * m,
+                       make_float4(xc[4 * m], xc[4 * m + 1], xc[4 * m + 2], xc[4 * m + 3]));
+      } else {
+#pragma unroll
+      for (int m = 0; m < 4; ++m)  // 32-byte stores (whole sectors)
+        st_stream_v8(dst + base + 32 * cc + 8 * m, __float_as_uint(xc[8 * m]), __float_as_uint(xc[8 * m + 1]),
+                     __float_as_uint(xc[8 * m + 2]), __float_as_uint(xc[8 * m + 3]), __float_as_uint(xc[8 * m + 4]),
+                     __float_as_uint(xc[8 * m + 5]), __float_as_uint(xc[8 * m + 6]), __float_as_uint(xc[8 * m + 7]));
+      }
+    } else if (!wide) {
 #pragma unroll
       for (int m = 0; m < 4; ++m) {
         uint4 v;
@@ -134,6 +144,14 @@ __device__ __forceinline__ void store_rowB_next(float (&x)[Geom<LOGN>::E], Tout*
         v.w = f32_to_bf16x2(xc[8 * m + 6], xc[8 * m + 7]);
         __stcs(reinterpret_cast<uint4*>(dst + base + 32 * cc + 8 * m), v);
       }
+    } else {
+#pragma unroll
+      for (int m = 0; m < 2; ++m)  // 32-byte stores (whole sectors)
+        st_stream_v8(dst + base + 32 * cc + 16 * m, f32_to_bf16x2(xc[16 * m], xc[16 * m + 1]),
+                     f32_to_bf16x2(xc[16 * m + 2], xc[16 * m + 3]), f32_to_bf16x2(xc[16 * m + 4], xc[16 * m + 5]),
+                     f32_to_bf16x2(xc[16 * m + 6], xc[16 * m + 7]), f32_to_bf16x2(xc[16 * m + 8], xc[16 * m + 9]),
+                     f32_to_bf16x2(xc[16 * m + 10], xc[16 * m + 11]), f32_to_bf16x2(xc[16 * m + 12], xc[16 * m + 13]),
+                     f32_to_bf16x2(xc[16 * m + 14], xc[16 * m + 15]));
     }
     next(cc);
   }

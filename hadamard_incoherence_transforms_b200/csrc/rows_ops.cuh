@@ -124,13 +124,15 @@ __device__ __forceinline__ void quant_rowB_next(float (&x)[Geom<LOGN>::E], const
     for (int cc = 0; cc < NCH; ++cc) mx[cc] = m;
   }
 
-  // 4- and 2-bit codes are packed and stored one 32-element chunk at a time
-  // (16 or 8 bytes per chunk); 3-bit chunks (12 bytes) are collected and
-  // stored as 16-byte vectors at the end.
+  // 4- and 2-bit codes are packed as each 32-element chunk is done and stored
+  // in 32-byte pieces (two 4-bit or four 2-bit chunks) when the thread's code
+  // run is 32-byte aligned, else per chunk; 3-bit chunks (12 bytes) are
+  // collected and stored as 16-byte vectors at the end.
   constexpr int NW = E * BITS / 32;  // packed words per thread
   constexpr int CW = BITS;           // packed words per 32-element chunk
-  uint32_t W[BITS == 3 ? NW : 1];
+  uint32_t W[BITS == 3 ? NW : 8];
   uint8_t* dst = a.codes + row * (int64_t(G::N) * BITS / 8) + int64_t(tau) * (E * BITS / 8);
+  const bool wide = (reinterpret_cast<uintptr_t>(dst) & 31) == 0;
   const int64_t spr = int64_t(G::N) >> lg;
   float s = 0.0f, ss = 0.0f, r = 0.0f, k = 1.0f;
 #pragma unroll
@@ -151,24 +153,35 @@ __device__ __forceinline__ void quant_rowB_next(float (&x)[Geom<LOGN>::E], const
     const float rr = s > 0.0f ? r : 0.0f;
     const float sx = s > 0.0f ? ss : 1.0f;
     if constexpr (BITS == 4) {
-      uint32_t w[4];
 #pragma unroll
       for (int v = 0; v < 4; ++v) {
         uint32_t ub[8];
         quant8<BITS>(xc + 8 * v, sx, rr, ub);
-        w[v] = pack4x8(ub);
+        W[4 * (cc & 1) + v] = pack4x8(ub);
       }
-      __stcs(reinterpret_cast<uint4*>(dst) + cc, make_uint4(w[0], w[1], w[2], w[3]));
+      // 32 bytes (two chunks) per store when aligned: whole sectors
+      if (NCH >= 2 && wide) {
+        if (cc & 1)
+          st_stream_v8(dst + 16 * (cc - 1), W[0], W[1], W[2], W[3], W[4], W[5], W[6], W[7]);
+      } else {
+        __stcs(reinterpret_cast<uint4*>(dst) + cc, make_uint4(W[4 * (cc & 1)], W[4 * (cc & 1) + 1],
+                                                             W[4 * (cc & 1) + 2], W[4 * (cc & 1) + 3]));
+      }
     } else if constexpr (BITS == 2) {
-      uint32_t w[2];
 #pragma unroll
       for (int v = 0; v < 2; ++v) {
         uint32_t ub[16];
         quant8<BITS>(xc + 16 * v, sx, rr, ub);
         quant8<BITS>(xc + 16 * v + 8, sx, rr, ub + 8);
-        w[v] = pack2x16(ub);
+        W[2 * (cc & 3) + v] = pack2x16(ub);
       }
-      __stcs(reinterpret_cast<uint2*>(dst) + cc, make_uint2(w[0], w[1]));
+      // 32 bytes (four chunks) per store when aligned
+      if (NCH >= 4 && wide) {
+        if ((cc & 3) == 3)
+          st_stream_v8(dst + 8 * (cc - 3), W[0], W[1], W[2], W[3], W[4], W[5], W[6], W[7]);
+      } else {
+        __stcs(reinterpret_cast<uint2*>(dst) + cc, make_uint2(W[2 * (cc & 3)], W[2 * (cc & 3) + 1]));
+      }
     } else {
       uint32_t ub[32];
 #pragma unroll
