@@ -226,10 +226,10 @@ cudaError_t launch_cols_full(int logm, int dt_in, int dt_out, const ColArgs& a, 
 // ---------------------------------------------------------------------------
 // Column transform for 1024 <= m <= 8192 with thread-block clusters.
 //
-// A cluster of CL = m / 1024 CTAs owns a strip of 16 adjacent columns over
-// all m rows; CTA c of the cluster holds rows [1024 c, 1024 c + 1024) of the
-// strip (64 KB fp32).  Row segments are 16 columns wide (32 B bf16 / 64 B
-// fp32), so global accesses are whole sectors.  Within a CTA a thread owns
+// A cluster of CL = m / 1024 CTAs owns a strip of 16 (bf16 source) or 8 (fp32
+// source) adjacent columns over all m rows; CTA c of the cluster holds rows
+// [1024 c, 1024 c + 1024) of the strip (64 or 32 KB fp32).  Row segments are
+// 32 bytes wide, so global accesses are whole sectors.  Within a CTA a thread owns
 // one 4-column quad and 32 rows: first rows tr + 32k (the register bits are
 // row bits 5..9), then, after one pass through shared memory, rows
 // 32 tr + r (row bits 0..4).  The CL row blocks (row bits 10 and up) are then
@@ -243,11 +243,22 @@ cudaError_t launch_cols_full(int logm, int dt_in, int dt_out, const ColArgs& a, 
 // copies (cp.async), so the loads of one strip overlap the arithmetic,
 // exchange and stores of the previous one.
 // ---------------------------------------------------------------------------
-constexpr int kQuads = 4;
-constexpr int kClusterThreads = kQuads * 32;
-// 16-byte chunk of (row, quad); bit 2 is xor-ed with row bit 5 so that rows
-// 32 apart (the phase-2 pattern) fall in different bank groups.
-__device__ __forceinline__ int cs_idx(int row, int q) { return (row * kQuads + q) ^ (((row >> 5) & 1) << 2); }
+// Quads (4-column groups) per strip: 4 for bf16 sources (16 columns, 32-byte
+// row segments), 2 for fp32 sources (8 columns, 32-byte row segments), so the
+// fp32 staging buffer stays small enough for three CTAs per SM.
+template <typename Tin>
+struct ClusterQuads {
+  static constexpr int QD = std::is_same<Tin, float>::value ? 2 : 4;
+  static constexpr int LQD = QD == 4 ? 2 : 1;
+};
+// 16-byte chunk of (row, quad); the bits above the quad index are xor-ed with
+// row bits 5.. so that rows 32 apart (the phase-2 pattern) fall in different
+// bank groups.
+template <int QD>
+__device__ __forceinline__ int cs_idx(int row, int q) {
+  constexpr int LQD = QD == 4 ? 2 : 1;
+  return (row * QD + q) ^ (((row >> 5) & (8 / QD - 1)) << LQD);
+}
 
 __device__ __forceinline__ void cp_async16(void* smem, const void* gmem) {
   asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(smem_u32(smem)), "l"(gmem) : "memory");
@@ -257,14 +268,18 @@ __device__ __forceinline__ void cp_async_wait_all() { asm volatile("cp.async.wai
 
 template <typename Tin>
 struct ClusterSmem {
-  static constexpr int SROW = 4 * kQuads * int(sizeof(Tin));  // staged bytes per row of a strip
-  static constexpr size_t WORK = size_t(1024) * kQuads * sizeof(float4);
+  static constexpr int QD = ClusterQuads<Tin>::QD;
+  static constexpr int THREADS = QD * 32;
+  static constexpr int SROW = 4 * QD * int(sizeof(Tin));  // staged bytes per row of a strip
+  static constexpr size_t WORK = size_t(1024) * QD * sizeof(float4);
   static constexpr size_t SMEM = WORK + size_t(1024) * SROW;
 };
 
 template <int CL, typename Tin, typename Tout>
-__global__ void __launch_bounds__(kClusterThreads) k_cols_cluster(const ColArgs a) {
+__global__ void __launch_bounds__(ClusterSmem<Tin>::THREADS) k_cols_cluster(const ColArgs a) {
   using SM = ClusterSmem<Tin>;
+  constexpr int kQuads = SM::QD;
+  constexpr int kClusterThreads = SM::THREADS;
   extern __shared__ float4 cs_smem[];  // [1024 rows][kQuads quads] fp32, then the staging rows
   uint8_t* stage = reinterpret_cast<uint8_t*>(cs_smem) + SM::WORK;
   namespace cg = cooperative_groups;
@@ -334,19 +349,19 @@ __global__ void __launch_bounds__(kClusterThreads) k_cols_cluster(const ColArgs 
     reg_stages<128, 2, 7>(x);  // row bits 5..9
 #pragma unroll
     for (int k = 0; k < 32; ++k)
-      cs_smem[cs_idx(tr + 32 * k, q)] = make_float4(x[4 * k], x[4 * k + 1], x[4 * k + 2], x[4 * k + 3]);
+      cs_smem[cs_idx<kQuads>(tr + 32 * k, q)] = make_float4(x[4 * k], x[4 * k + 1], x[4 * k + 2], x[4 * k + 3]);
     __syncthreads();
     // phase 2: rows 32 tr + r
 #pragma unroll
     for (int r = 0; r < 32; ++r) {
-      const float4 v = cs_smem[cs_idx(32 * tr + r, q)];
+      const float4 v = cs_smem[cs_idx<kQuads>(32 * tr + r, q)];
       x[4 * r] = v.x; x[4 * r + 1] = v.y; x[4 * r + 2] = v.z; x[4 * r + 3] = v.w;
     }
     reg_stages<128, 2, 7>(x);  // row bits 0..4
     __syncthreads();           // every phase-2 read is done before the writes
 #pragma unroll
     for (int r = 0; r < 32; ++r)
-      cs_smem[cs_idx(32 * tr + r, q)] = make_float4(x[4 * r], x[4 * r + 1], x[4 * r + 2], x[4 * r + 3]);
+      cs_smem[cs_idx<kQuads>(32 * tr + r, q)] = make_float4(x[4 * r], x[4 * r + 1], x[4 * r + 2], x[4 * r + 3]);
     cluster.sync();  // all blocks of the strip are in shared memory
     // phase 3: this CTA combines rows (c', row_low) for row_low in its share
     Tout* dst = static_cast<Tout*>(a.y) + strip * 4 * kQuads + 4 * q;
@@ -357,7 +372,7 @@ __global__ void __launch_bounds__(kClusterThreads) k_cols_cluster(const ColArgs 
 #pragma unroll
       for (int c = 0; c < CL; ++c) {
         const float4* rem = cluster.map_shared_rank(cs_smem, c);
-        const float4 w = rem[cs_idx(row_low, q)];
+        const float4 w = rem[cs_idx<kQuads>(row_low, q)];
         v[4 * c] = w.x; v[4 * c + 1] = w.y; v[4 * c + 2] = w.z; v[4 * c + 3] = w.w;
       }
       if constexpr (CL > 1) reg_stages<4 * CL, 2, 2 + (CL == 2 ? 1 : (CL == 4 ? 2 : 3))>(v);
@@ -385,9 +400,9 @@ static cudaError_t launch_cluster_t(const ColArgs& a, cudaStream_t st) {
   static std::atomic<unsigned long long> done{0};
   cudaError_t e = set_smem_attr(kern, SM::SMEM, done);
   if (e != cudaSuccess) return e;
-  const int64_t strips = a.cols / (4 * kQuads);
+  const int64_t strips = a.cols / (4 * SM::QD);
   cudaLaunchConfig_t cfg = {};
-  cfg.blockDim = dim3(kClusterThreads);
+  cfg.blockDim = dim3(SM::THREADS);
   cfg.dynamicSmemBytes = SM::SMEM;
   cfg.stream = st;
   cudaLaunchAttribute attr[1];
@@ -425,7 +440,7 @@ static cudaError_t launch_cluster_cl(int dt_in, int dt_out, const ColArgs& a, cu
 }
 
 cudaError_t launch_cols_cluster(int logm, int dt_in, int dt_out, const ColArgs& a, cudaStream_t st) {
-  if (a.cols % (4 * kQuads) != 0 || a.cols / (4 * kQuads) > 0x7fffffffLL / 8) return cudaErrorInvalidValue;
+  if (a.cols % 16 != 0 || a.cols / 8 > 0x7fffffffLL / 8) return cudaErrorInvalidValue;
   switch (logm) {
     case 10: return launch_cluster_cl<1>(dt_in, dt_out, a, st);
     case 11: return launch_cluster_cl<2>(dt_in, dt_out, a, st);
