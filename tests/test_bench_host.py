@@ -1,0 +1,41 @@
+"""Host-side logic of bench.py that needs no GPU: the peak used as the
+roofline denominator, and the rule that DRAM traffic from a committed ncu
+capture is reported only while the kernel sources match the capture."""
+import json
+import os
+
+import bench
+
+
+def test_measured_peak_prefers_the_driver_file(tmp_path, monkeypatch):
+    monkeypatch.setattr(bench, "ROOT", str(tmp_path))
+    assert bench.measured_peaks() == (bench.FALLBACK_HBM_GBS, "fallback")
+    (tmp_path / "MEASURED_PEAKS.json").write_text(json.dumps({"hbm_gbs": 1234.5}))
+    assert bench.measured_peaks() == (1234.5, "measured")
+
+
+def test_traffic_is_reported_only_for_matching_sources(tmp_path, monkeypatch):
+    real_root = bench.ROOT
+    digest = bench.source_digest()
+    assert len(digest) == 16 and digest == bench.source_digest()  # stable for the same sources
+    prof = tmp_path / "profiles"
+    prof.mkdir()
+    monkeypatch.setattr(bench, "ROOT", str(tmp_path))
+    monkeypatch.setattr(bench, "source_digest", lambda: digest)
+    rec = {"k": {"dram_bytes_per_launch": 42.0, "source_digest": digest}}
+    (prof / "traffic.json").write_text(json.dumps(rec))
+    assert bench.read_profile_traffic("k") == 42.0
+    assert bench.read_profile_traffic("other") is None
+    rec["k"]["source_digest"] = "0" * 16
+    (prof / "traffic.json").write_text(json.dumps(rec))
+    assert bench.read_profile_traffic("k") is None
+    monkeypatch.setattr(bench, "ROOT", real_root)
+
+
+def test_committed_traffic_record_names_the_headline_kernel():
+    path = os.path.join(bench.ROOT, "profiles", "traffic.json")
+    with open(path) as f:
+        rec = json.load(f)
+    assert "k_rows_stream<12,float,float,EPI_QUANT,4>" in rec
+    r = rec["k_rows_stream<12,float,float,EPI_QUANT,4>"]
+    assert r["dram_bytes_per_launch"] == r["dram_read"] + r["dram_write"]
