@@ -11,7 +11,7 @@ sets whose total exceeds 4x the L2 size, so no step reads its input from L2.
 Throughput counts algorithmic bytes only (input read once, codes and scales
 written once).  Prints one JSON line (rank 0).
 
---impl reference times the CPU oracle (the reference arm of this build) on a
+--impl reference times the CPU oracle (the reference arm) on a
 bounded sample of the same workload per step.
 """
 from __future__ import annotations
