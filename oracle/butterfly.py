@@ -22,10 +22,19 @@ Convention chosen (the pages leave it open):
 With every block equal to H_b / sqrt(b) this convention gives exactly
 H_d / sqrt(d) because the Sylvester matrices satisfy H_a (x) H_b = H_ab.
 
+The randomized transform for lengths that are not powers of two (HARP
+explainer, technical summary §2.1: stride stages for any factorization of d,
+e.g. d = 5120 = 8 * 8 * 8 * 5 * 2) is read the same way as the power-of-two
+RHT: y = R diag(s) x, with Hadamard blocks H_b / sqrt(b) for the power-of-two
+radices and orthogonal mixers for the others; its inverse is
+x = diag(s) R^T y.
+
 Pinned by tests/test_oracle_butterfly.py: a pure-Python index-loop evaluation
 of the definition on tiny schedules, the all-Hadamard case against the
 popcount formula for H_d, a single full-width stage against a dense matrix
-product, orthogonality of the dense R, and R^T R = I.
+product, orthogonality of the dense R, and R^T R = I; the mixed-radix RHT
+against the dense Sylvester RHT when every radix is a power of two, norm
+preservation with a radix-5 mixer, and inverse after forward.
 """
 from __future__ import annotations
 
@@ -85,3 +94,14 @@ def dense(radices, blocks, transpose: bool = False) -> np.ndarray:
 def two_sided(w, radices_in, blocks_in, radices_out, blocks_out) -> np.ndarray:
     """W' = R_out W R_in^T: R_in along every row, R_out along every column."""
     return apply_stages_cols(apply_stages(w, radices_in, blocks_in), radices_out, blocks_out)
+
+
+def rht_mixed(x, signs, radices, blocks) -> np.ndarray:
+    """y = R diag(s) x for every row of x (signs applied first)."""
+    x = np.asarray(x, dtype=np.float64) * np.asarray(signs, dtype=np.float64)
+    return apply_stages(x, radices, blocks)
+
+
+def irht_mixed(y, signs, radices, blocks) -> np.ndarray:
+    """x = diag(s) R^T y for every row of y (the inverse of rht_mixed)."""
+    return apply_stages(y, radices, blocks, transpose=True) * np.asarray(signs, dtype=np.float64)

@@ -33,6 +33,7 @@ WORKLOADS = {
     "two_sided_butterfly": 3,
     "two_sided_lowbit": 4,
     "wht_adapter": 5,
+    "mixed_rht_int4": 6,
 }
 
 
@@ -107,6 +108,29 @@ def two_sided_butterfly(rows: int = 4096, d: int = 14336,
     blocks_out = [seeded_orthogonal_blocks(rbo, rows // b, b) for b in radices_out]
     return {"x_bf16": to_bf16_bits(x), "radices_in": tuple(radices_in), "blocks_in": blocks_in,
             "radices_out": tuple(radices_out), "blocks_out": blocks_out}
+
+
+def hadamard_block(b: int) -> np.ndarray:
+    """The normalized Sylvester Hadamard H_b / sqrt(b) (b a power of two), as a
+    [1, b, b] shared block: entry (i, j) is (-1)^popcount(i & j) / sqrt(b)."""
+    i = np.arange(b)
+    par = np.vectorize(lambda v: bin(int(v)).count("1") & 1)(i[:, None] & i[None, :])
+    return ((1.0 - 2.0 * par) / np.sqrt(b)).astype(np.float32)[None]
+
+
+def mixed_rht_int4(rows: int = 4096, d: int = 5120, radices=(8, 8, 8, 5, 2), seed: int | None = None) -> dict:
+    """Rows of length d = prod(radices) (not a power of two), N(0, 0.02) with
+    0.1 % outliers x 50; Rademacher signs; Hadamard blocks for the power-of-two
+    radices and one seeded orthogonal block per group for the others."""
+    if int(np.prod(radices)) != d:
+        raise ValueError("radices must multiply to d")
+    rv, rp, rs, rb = streams("mixed_rht_int4", 4, seed)
+    x = (rv.standard_normal((rows, d)) * 0.02).astype(np.float32)
+    pos = distinct_positions(rp, rows * d, int(round(0.001 * rows * d)))
+    x.reshape(-1)[pos] *= np.float32(50.0)
+    blocks = [hadamard_block(b) if (b & (b - 1)) == 0 else seeded_orthogonal_blocks(rb, d // b, b) for b in radices]
+    return {"x": x, "signs": rademacher(rs, d), "radices": tuple(radices), "blocks": blocks, "bits": 4,
+            "group": 128}
 
 
 def two_sided_lowbit(rows: int = 8192, n: int = 8192, seed: int | None = None) -> dict:
