@@ -279,7 +279,7 @@ def two_sided_lowbit(dev, l2_bytes, host_only=False, bits=3):
     q_b = rows * n * bits // 8 + rows * (n // group) * 4
     w.bytes = rows * n * 2 + q_b + q_b + rows * n * 4
     w.h2d, w.d2h = rows * n * 2, rows * n * 4
-    w.kernels_per_step = 6
+    w.kernels_per_step = 4  # column pass + row quantize; row dequantize + column pass
     w.kernel_key = "k_cols_cluster<8,bf16,float>"
 
     def oracle(r0, r1):
@@ -377,7 +377,7 @@ def two_sided_butterfly(dev, l2_bytes, host_only=False):
     w.desc = "bf16 4096x14336: R_in (7,16,16,8) along rows then R_out (16,16,16) along columns"
     w.bytes = rows * n * 4
     w.h2d = w.d2h = rows * n * 2
-    w.kernels_per_step = 7
+    w.kernels_per_step = 4  # two row passes (R_in) and two column passes (R_out)
     w.kernel_key = "k_bfly_pass"
 
     def oracle(r0, r1):
