@@ -20,13 +20,15 @@ Sources (page title, section):
   fast, O(d log d), exactly orthogonal), §2.1 (mixed-radix schedule of
   stride-based block-diagonal orthogonal stages), §2.2 (normalized Sylvester
   Hadamard as the fixed mixer; zero-initialised HARP recovers the RHT), §5
-  (exact change of basis, two-sided processor).
+  (exact change of basis, two-sided processor); §2.2 also gives the learnable
+  blocks Q(theta) G (Givens / Cayley) and §2.4 their int8 storage.
 * QWHA: Quantization-Aware Walsh-Hadamard Adaptation for Parameter-Efficient
   Fine-Tuning on Large Language Models -- technical summary §2.1 (single
   transform adapter dW = F H^-1, F sparse from a value vector c and an index
-  list E; WHT kernel of +-1 entries, add/subtract only), §4 (scatter
-  operations).
+  list E; WHT kernel of +-1 entries, add/subtract only; the two-transform form
+  H'^-1 F H^-1), §2.2 (AdaAlloc budget split and per-channel top-k,
+  least-squares Refinement), §4 (scatter operations).
 
 Parity status of each function is stated in its module header.
 """
-from . import hadamard, quant, butterfly, sparse  # noqa: F401
+from . import hadamard, quant, butterfly, sparse, harp, qwha  # noqa: F401

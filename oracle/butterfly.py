@@ -40,6 +40,8 @@ from __future__ import annotations
 
 import numpy as np
 
+from .hadamard import is_pow2, sylvester
+
 
 def strides(radices) -> list[int]:
     out, acc = [], 1
@@ -94,6 +96,20 @@ def dense(radices, blocks, transpose: bool = False) -> np.ndarray:
 def two_sided(w, radices_in, blocks_in, radices_out, blocks_out) -> np.ndarray:
     """W' = R_out W R_in^T: R_in along every row, R_out along every column."""
     return apply_stages_cols(apply_stages(w, radices_in, blocks_in), radices_out, blocks_out)
+
+
+def rht_stage_blocks(radices, mixers=None) -> list[np.ndarray]:
+    """Stage blocks of the mixed-radix RHT: the shared [1, b, b] block H_b / sqrt(b)
+    for a power-of-two radix, the given orthogonal blocks mixers[b] otherwise."""
+    out = []
+    for b in (int(v) for v in radices):
+        if is_pow2(b):
+            out.append((sylvester(b) / np.sqrt(b))[None])
+        elif mixers is None or b not in mixers:
+            raise ValueError(f"radix {b} is not a power of two: its orthogonal blocks must be given")
+        else:
+            out.append(np.asarray(mixers[b], dtype=np.float64))
+    return out
 
 
 def rht_mixed(x, signs, radices, blocks) -> np.ndarray:

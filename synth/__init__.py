@@ -20,6 +20,18 @@ Recipes (one seed per workload, child streams per quantity):
   multiplied by 100; row and column Rademacher signs.
 * ``wht_adapter``       [32, 4096, 64] fp32 values ~ N(0, (1e-3)^2) and int32
   column indices: 64 distinct uniform columns per row, sorted ascending.
+* ``mixed_rht_int4``    fp32 [4096, 5120] as the weight recipe; radices
+  (8, 8, 8, 5, 2): one seeded orthogonal block per group for radix 5 (the
+  power-of-two radices use Hadamard blocks, which are not inputs).
+* ``harp_rotation``     fp32 [4096, d] as the weight recipe; Rademacher signs;
+  per stage and group the learnable parameters ~ N(0, 0.05^2) (a small
+  refinement around the zero start); d = 4096 with radices (16, 16, 16), or
+  d = 5120 with (8, 8, 8, 5, 2) and one seeded orthogonal mixer for radix 5.
+* ``qwha_init``         fp32 weight [4096, 4096] as the weight recipe with
+  Rademacher signs (its quantization error is what the adapter targets);
+  activations fp32 [4096, 512] ~ N(0, 1) with 1 % of input channels (rounded)
+  multiplied by 20; a budget of 64 parameters per row on average with at
+  least 1 per row.
 """
 from __future__ import annotations
 
@@ -34,6 +46,8 @@ WORKLOADS = {
     "two_sided_lowbit": 4,
     "wht_adapter": 5,
     "mixed_rht_int4": 6,
+    "harp_rotation": 7,
+    "qwha_init": 8,
 }
 
 
@@ -110,27 +124,54 @@ def two_sided_butterfly(rows: int = 4096, d: int = 14336,
             "radices_out": tuple(radices_out), "blocks_out": blocks_out}
 
 
-def hadamard_block(b: int) -> np.ndarray:
-    """The normalized Sylvester Hadamard H_b / sqrt(b) (b a power of two), as a
-    [1, b, b] shared block: entry (i, j) is (-1)^popcount(i & j) / sqrt(b)."""
-    i = np.arange(b)
-    par = np.vectorize(lambda v: bin(int(v)).count("1") & 1)(i[:, None] & i[None, :])
-    return ((1.0 - 2.0 * par) / np.sqrt(b)).astype(np.float32)[None]
-
-
 def mixed_rht_int4(rows: int = 4096, d: int = 5120, radices=(8, 8, 8, 5, 2), seed: int | None = None) -> dict:
     """Rows of length d = prod(radices) (not a power of two), N(0, 0.02) with
-    0.1 % outliers x 50; Rademacher signs; Hadamard blocks for the power-of-two
-    radices and one seeded orthogonal block per group for the others."""
+    0.1 % outliers x 50; Rademacher signs; for every radix that is not a power
+    of two, one seeded orthogonal block per group ([d / b, b, b] under key b).
+    The power-of-two radices carry no input: their blocks are the Hadamard ones."""
     if int(np.prod(radices)) != d:
         raise ValueError("radices must multiply to d")
     rv, rp, rs, rb = streams("mixed_rht_int4", 4, seed)
     x = (rv.standard_normal((rows, d)) * 0.02).astype(np.float32)
     pos = distinct_positions(rp, rows * d, int(round(0.001 * rows * d)))
     x.reshape(-1)[pos] *= np.float32(50.0)
-    blocks = [hadamard_block(b) if (b & (b - 1)) == 0 else seeded_orthogonal_blocks(rb, d // b, b) for b in radices]
-    return {"x": x, "signs": rademacher(rs, d), "radices": tuple(radices), "blocks": blocks, "bits": 4,
+    mixers = {b: seeded_orthogonal_blocks(rb, d // b, b) for b in sorted(set(radices)) if b & (b - 1)}
+    return {"x": x, "signs": rademacher(rs, d), "radices": tuple(radices), "mixers": mixers, "bits": 4,
             "group": 128}
+
+
+def harp_rotation(rows: int = 4096, d: int = 4096, radices=(16, 16, 16), theta_std: float = 0.05,
+                  seed: int | None = None) -> dict:
+    """Weights, signs and per-stage learnable parameters [d / b_t, P(b_t)] with
+    P(1) = 0, P(2) = 1 and P(b) = b (b - 1) / 2; one seeded orthogonal mixer per
+    radix that is not a power of two."""
+    radices = tuple(int(b) for b in radices)
+    if int(np.prod(radices)) != d:
+        raise ValueError("radices must multiply to d")
+    rv, rp, rs, rt, rm = streams("harp_rotation", 5, seed)
+    x = (rv.standard_normal((rows, d)) * 0.02).astype(np.float32)
+    pos = distinct_positions(rp, rows * d, int(round(0.001 * rows * d)))
+    x.reshape(-1)[pos] *= np.float32(50.0)
+    counts = [0 if b == 1 else 1 if b == 2 else b * (b - 1) // 2 for b in radices]
+    thetas = [(rt.standard_normal((d // b, p)) * theta_std).astype(np.float32) for b, p in zip(radices, counts)]
+    base = {b: seeded_orthogonal_blocks(rm, 1, b)[0] for b in sorted(set(radices)) if b & (b - 1)}
+    return {"x": x, "signs": rademacher(rs, d), "radices": radices, "thetas": thetas, "base_mixers": base,
+            "bits": 4, "group": 128}
+
+
+def qwha_init(rows: int = 4096, n: int = 4096, tokens: int = 512, per_row: int = 64, k_min: int = 1,
+              seed: int | None = None) -> dict:
+    """Weights to be quantized, Rademacher signs for the rotated quantizer,
+    synthetic activations with outlier input channels, and the parameter budget."""
+    rv, rp, rs, rx, rc = streams("qwha_init", 5, seed)
+    w = (rv.standard_normal((rows, n)) * 0.02).astype(np.float32)
+    pos = distinct_positions(rp, rows * n, int(round(0.001 * rows * n)))
+    w.reshape(-1)[pos] *= np.float32(50.0)
+    x = rx.standard_normal((n, tokens)).astype(np.float32)
+    hot = distinct_positions(rc, n, int(round(0.01 * n)))
+    x[hot, :] *= np.float32(20.0)
+    return {"w": w, "signs": rademacher(rs, n), "x": x, "budget": per_row * rows, "k_min": k_min,
+            "bits": 4, "group": 128, "outlier_channels": hot}
 
 
 def two_sided_lowbit(rows: int = 8192, n: int = 8192, seed: int | None = None) -> dict:

@@ -8,6 +8,7 @@ import synth
 from oracle import butterfly as ob
 from oracle import hadamard as oh
 from tests._parity import assert_close, host, to_gpu_bf16, to_gpu_f32
+from tests.test_oracle_hadamard import popcount_hadamard
 
 pytestmark = pytest.mark.gpu
 
@@ -49,7 +50,7 @@ def test_shared_blocks_and_bf16():
 
 def test_hadamard_blocks_recover_the_rht():
     radices = (16, 16, 16)
-    h16 = (oh.sylvester(16) / 4.0).astype(np.float32)
+    h16 = (popcount_hadamard(16) / 4.0).astype(np.float32)     # input blocks, not from the oracle
     blocks = [np.broadcast_to(h16, (256, 16, 16)).copy() for _ in radices]
     x = np.random.default_rng(2).standard_normal((9, 4096)).astype(np.float32)
     y = hit.butterfly_apply(to_gpu_f32(x), radices, [to_gpu_f32(b) for b in blocks])

@@ -122,25 +122,22 @@ def test_columns_direction():
 def test_mixed_rht_equals_dense_sylvester_rht_for_power_of_two_radices():
     """With Hadamard blocks on every power-of-two radix the mixed-radix RHT is
     the RHT of the dense Sylvester path: (x * s) @ H_d / sqrt(d)."""
-    from oracle import hadamard as oh
-    from synth import hadamard_block
-
     rng = np.random.default_rng(5)
     radices = (4, 2, 8)
     d = 64
     x = rng.standard_normal((3, d))
     s = np.where(rng.random(d) < 0.5, -1, 1).astype(np.int8)
-    y = ob.rht_mixed(x, s, radices, [hadamard_block(b) for b in radices])
-    assert np.allclose(y, oh.rht_rows(x, s), atol=1e-12)
+    y = ob.rht_mixed(x, s, radices, ob.rht_stage_blocks(radices))
+    assert np.allclose(y, (x * s) @ popcount_hadamard(d) / 8.0, atol=1e-12)
+    for b, blk in zip(radices, ob.rht_stage_blocks(radices)):
+        assert np.array_equal(blk[0], popcount_hadamard(b) / np.sqrt(b))
 
 
 def test_mixed_rht_with_radix_five_preserves_norms_and_inverts():
-    from synth import hadamard_block
-
     rng = np.random.default_rng(6)
     radices = (8, 5, 2)
     d = 80
-    blocks = [hadamard_block(8), seeded_orthogonal_blocks(rng, d // 5, 5), hadamard_block(2)]
+    blocks = ob.rht_stage_blocks(radices, {5: seeded_orthogonal_blocks(rng, d // 5, 5)})
     x = rng.standard_normal((4, d))
     s = np.where(rng.random(d) < 0.5, -1, 1).astype(np.int8)
     y = ob.rht_mixed(x, s, radices, blocks)
@@ -158,6 +155,8 @@ def test_mixed_rht_synthetic_recipe():
 
     d = mixed_rht_int4(rows=8)
     assert d["x"].shape == (8, 5120) and d["radices"] == (8, 8, 8, 5, 2)
-    assert [b.shape for b in d["blocks"]] == [(1, 8, 8), (1, 8, 8), (1, 8, 8), (1024, 5, 5), (1, 2, 2)]
-    y = ob.rht_mixed(d["x"], d["signs"], d["radices"], d["blocks"])
+    assert list(d["mixers"]) == [5] and d["mixers"][5].shape == (1024, 5, 5)
+    blocks = ob.rht_stage_blocks(d["radices"], d["mixers"])
+    assert [b.shape for b in blocks] == [(1, 8, 8), (1, 8, 8), (1, 8, 8), (1024, 5, 5), (1, 2, 2)]
+    y = ob.rht_mixed(d["x"], d["signs"], d["radices"], blocks)
     assert np.allclose(np.linalg.norm(y, axis=1), np.linalg.norm(d["x"].astype(np.float64), axis=1), rtol=1e-5)

@@ -42,3 +42,22 @@ def test_two_sided_recipe_small():
     d = synth.two_sided_lowbit(rows=64, n=128)
     assert d["x_bf16"].dtype == np.uint16 and d["x_bf16"].shape == (64, 128)
     assert d["row_signs"].shape == (128,) and d["col_signs"].shape == (64,)
+
+
+def test_harp_recipe_small():
+    a = synth.harp_rotation(rows=8, d=64, radices=(4, 4, 4))
+    b = synth.harp_rotation(rows=8, d=64, radices=(4, 4, 4))
+    assert all(np.array_equal(p, q) for p, q in zip(a["thetas"], b["thetas"]))
+    assert [t.shape for t in a["thetas"]] == [(16, 6)] * 3 and a["base_mixers"] == {}
+    c = synth.harp_rotation(rows=8, d=80, radices=(8, 5, 2))
+    assert [t.shape for t in c["thetas"]] == [(10, 28), (16, 10), (40, 1)]
+    g = c["base_mixers"][5].astype(np.float64)
+    np.testing.assert_allclose(g.T @ g, np.eye(5), atol=1e-6)
+    assert abs(float(np.std(np.concatenate([t.ravel() for t in c["thetas"]]))) - 0.05) < 0.01
+
+
+def test_qwha_recipe_small():
+    d = synth.qwha_init(rows=32, n=128, tokens=16, per_row=8)
+    assert d["w"].shape == (32, 128) and d["x"].shape == (128, 16) and d["budget"] == 256
+    assert len(d["outlier_channels"]) == round(0.01 * 128)
+    assert np.all(np.abs(d["x"][d["outlier_channels"]]).mean(axis=1) > 5)
