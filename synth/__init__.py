@@ -21,8 +21,8 @@ Recipes (one seed per workload, child streams per quantity):
 * ``wht_adapter``       [32, 4096, 64] fp32 values ~ N(0, (1e-3)^2) and int32
   column indices: 64 distinct uniform columns per row, sorted ascending.
 * ``mixed_rht_int4``    fp32 [4096, 5120] as the weight recipe; radices
-  (8, 8, 8, 5, 2): one seeded orthogonal block per group for radix 5 (the
-  power-of-two radices use Hadamard blocks, which are not inputs).
+  (8, 8, 8, 5, 2): one seeded orthogonal 5 x 5 mixer shared by every group
+  (the power-of-two radices use Hadamard blocks, which are not inputs).
 * ``harp_rotation``     fp32 [4096, d] as the weight recipe; Rademacher signs;
   per stage and group the learnable parameters ~ N(0, 0.05^2) (a small
   refinement around the zero start); d = 4096 with radices (16, 16, 16), or
@@ -126,16 +126,17 @@ def two_sided_butterfly(rows: int = 4096, d: int = 14336,
 
 def mixed_rht_int4(rows: int = 4096, d: int = 5120, radices=(8, 8, 8, 5, 2), seed: int | None = None) -> dict:
     """Rows of length d = prod(radices) (not a power of two), N(0, 0.02) with
-    0.1 % outliers x 50; Rademacher signs; for every radix that is not a power
-    of two, one seeded orthogonal block per group ([d / b, b, b] under key b).
-    The power-of-two radices carry no input: their blocks are the Hadamard ones."""
+    0.1 % outliers x 50; Rademacher signs; for every radix b that is not a power
+    of two, one seeded orthogonal mixer shared by all groups ([1, b, b] under
+    key b).  The power-of-two radices carry no input: their blocks are the
+    Hadamard ones."""
     if int(np.prod(radices)) != d:
         raise ValueError("radices must multiply to d")
     rv, rp, rs, rb = streams("mixed_rht_int4", 4, seed)
     x = (rv.standard_normal((rows, d)) * 0.02).astype(np.float32)
     pos = distinct_positions(rp, rows * d, int(round(0.001 * rows * d)))
     x.reshape(-1)[pos] *= np.float32(50.0)
-    mixers = {b: seeded_orthogonal_blocks(rb, d // b, b) for b in sorted(set(radices)) if b & (b - 1)}
+    mixers = {b: seeded_orthogonal_blocks(rb, 1, b) for b in sorted(set(radices)) if b & (b - 1)}
     return {"x": x, "signs": rademacher(rs, d), "radices": tuple(radices), "mixers": mixers, "bits": 4,
             "group": 128}
 

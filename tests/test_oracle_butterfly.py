@@ -155,8 +155,33 @@ def test_mixed_rht_synthetic_recipe():
 
     d = mixed_rht_int4(rows=8)
     assert d["x"].shape == (8, 5120) and d["radices"] == (8, 8, 8, 5, 2)
-    assert list(d["mixers"]) == [5] and d["mixers"][5].shape == (1024, 5, 5)
+    assert list(d["mixers"]) == [5] and d["mixers"][5].shape == (1, 5, 5)
     blocks = ob.rht_stage_blocks(d["radices"], d["mixers"])
-    assert [b.shape for b in blocks] == [(1, 8, 8), (1, 8, 8), (1, 8, 8), (1024, 5, 5), (1, 2, 2)]
+    assert [b.shape for b in blocks] == [(1, 8, 8), (1, 8, 8), (1, 8, 8), (1, 5, 5), (1, 2, 2)]
     y = ob.rht_mixed(d["x"], d["signs"], d["radices"], blocks)
     assert np.allclose(np.linalg.norm(y, axis=1), np.linalg.norm(d["x"].astype(np.float64), axis=1), rtol=1e-5)
+
+
+@pytest.mark.parametrize("radices", [(8, 5, 2), (2, 3, 4), (5, 4), (3, 3, 2)])
+def test_shared_blocks_give_the_kronecker_product(radices):
+    """With one block per stage, R = B_0 (x) B_1 (x) ... (x) B_{m-1} (digit 0 most
+    significant, the row-major convention of np.kron), so the order of the stages
+    does not matter."""
+    rng = np.random.default_rng(sum(radices))
+    blocks = [rng.standard_normal((1, b, b)) for b in radices]
+    want = blocks[0][0]
+    for blk in blocks[1:]:
+        want = np.kron(want, blk[0])
+    np.testing.assert_allclose(ob.dense(radices, blocks), want, rtol=0, atol=1e-12)
+
+
+def test_mixed_rht_is_harp_at_zero_parameters():
+    """The mixed-radix RHT with one shared QR mixer is HARP's transform at theta = 0."""
+    from oracle import harp as oha
+    from synth import mixed_rht_int4
+
+    d = mixed_rht_int4(rows=3, d=80, radices=(8, 5, 2))
+    thetas = [np.zeros((80 // b, oha.n_params(b))) for b in d["radices"]]
+    y_harp = oha.forward(d["x"], d["signs"], d["radices"], thetas, {5: d["mixers"][5][0]})
+    y_rht = ob.rht_mixed(d["x"], d["signs"], d["radices"], ob.rht_stage_blocks(d["radices"], d["mixers"]))
+    np.testing.assert_allclose(y_harp, y_rht, rtol=0, atol=1e-14)
