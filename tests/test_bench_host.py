@@ -39,3 +39,27 @@ def test_committed_traffic_record_names_the_headline_kernel():
     assert "k_rows_stream<12,float,float,EPI_QUANT,4>" in rec
     r = rec["k_rows_stream<12,float,float,EPI_QUANT,4>"]
     assert r["dram_bytes_per_launch"] == r["dram_read"] + r["dram_write"]
+
+
+def test_reference_arm_prints_one_contract_line(capsys):
+    """The reference arm (the oracle on host cores) runs without a GPU and prints
+    the JSON line with the keys the driver reads."""
+    assert bench.main(["--impl", "reference", "--steps", "3", "--warmup", "3"]) == 0
+    lines = [l for l in capsys.readouterr().out.splitlines() if l.strip()]
+    assert len(lines) == 1
+    d = json.loads(lines[0])
+    for key in ("metric", "value", "unit", "n_gpus", "steps", "warmup", "ms_per_step", "higher_is_better",
+                "scaling", "vs_baseline", "dtype", "data", "config", "cpu_baseline", "e2e"):
+        assert key in d, key
+    assert d["impl"] == "reference" and d["steps"] == 3 and d["warmup"] == 3 and d["value"] > 0
+    assert d["cpu_baseline"]["kind"] == "oracle" and d["cpu_baseline"]["value"] == d["value"]
+    assert d["e2e"] == {"value": d["value"], "unit": d["unit"], "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}
+    assert "workload" in d["config"]
+
+
+def test_reference_arm_is_silent_on_other_ranks(capsys):
+    class Args:
+        workload, steps, warmup = "weight_rht_int4", 3, 3
+
+    assert bench.run_reference(Args(), 2, 1) == 0
+    assert capsys.readouterr().out == ""
