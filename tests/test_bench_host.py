@@ -63,3 +63,43 @@ def test_reference_arm_is_silent_on_other_ranks(capsys):
 
     assert bench.run_reference(Args(), 2, 1) == 0
     assert capsys.readouterr().out == ""
+
+
+def test_clock_sampler_with_a_fake_nvml(monkeypatch):
+    """The sampler reads SM clocks and throttle reasons through NVML; a fake
+    module stands in for it on a machine without a GPU."""
+    import sys
+    import time
+    import types
+
+    state = {"n": 0}
+    fake = types.SimpleNamespace(
+        NVML_CLOCK_SM=1,
+        nvmlInit=lambda: None,
+        nvmlDeviceGetHandleByIndex=lambda i: ("h", i),
+        nvmlDeviceGetMaxClockInfo=lambda h, kind: 1965,
+    )
+
+    def clock(h, kind):
+        state["n"] += 1
+        return 1965 if state["n"] % 3 else 1800
+
+    fake.nvmlDeviceGetClockInfo = clock
+    fake.nvmlDeviceGetCurrentClocksEventReasons = lambda h: 0x1 | 0x4   # idle (ignored) + power cap
+    monkeypatch.setitem(sys.modules, "pynvml", fake)
+    monkeypatch.delenv("CUDA_VISIBLE_DEVICES", raising=False)
+    with bench.ClockSampler(0) as clk:
+        time.sleep(0.05)
+    out = clk.summary()
+    assert out["sm_max_mhz"] == 1965 and out["samples"] >= 5
+    assert out["sm_mhz"] == 1965
+    assert out["reasons"] == ["sw_power_cap"]
+
+
+def test_clock_sampler_without_nvml(monkeypatch):
+    import sys
+
+    monkeypatch.setitem(sys.modules, "pynvml", None)   # import fails
+    with bench.ClockSampler(0) as clk:
+        pass
+    assert clk.summary() == {"sm_mhz": None, "sm_max_mhz": None, "reasons": [], "samples": 0}
