@@ -137,26 +137,28 @@ class ClockSampler:
 
 def read_profile_traffic(kernel_key: str):
     """Per-launch DRAM bytes of `kernel_key` from profiles/traffic.json, if the
-    recorded source digest matches the current kernel sources (else None)."""
+    digest of the sources the record names (the kernel's translation unit and
+    the build script) still matches (else None)."""
     path = os.path.join(ROOT, "profiles", "traffic.json")
     try:
         with open(path) as f:
             rec = json.load(f).get(kernel_key)
-        if rec and rec.get("source_digest") == source_digest():
+        if rec and rec.get("source_digest") == source_digest(rec["sources"]):
             return float(rec["dram_bytes_per_launch"])
     except Exception:
         pass
     return None
 
 
-def source_digest() -> str:
+def source_digest(sources) -> str:
+    """sha256 prefix over the named files (paths relative to the package directory)."""
     import hashlib
 
     h = hashlib.sha256()
-    csrc = os.path.join(ROOT, "hadamard_incoherence_transforms_b200", "csrc")
-    for f in sorted(os.listdir(csrc)):
-        with open(os.path.join(csrc, f), "rb") as fh:
-            h.update(f.encode() + fh.read())
+    pkg = os.path.join(ROOT, "hadamard_incoherence_transforms_b200")
+    for rel in sources:
+        with open(os.path.join(pkg, rel), "rb") as fh:
+            h.update(rel.encode() + fh.read())
     return h.hexdigest()[:16]
 
 

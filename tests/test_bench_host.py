@@ -15,21 +15,27 @@ def test_measured_peak_prefers_the_driver_file(tmp_path, monkeypatch):
 
 
 def test_traffic_is_reported_only_for_matching_sources(tmp_path, monkeypatch):
-    real_root = bench.ROOT
-    digest = bench.source_digest()
-    assert len(digest) == 16 and digest == bench.source_digest()  # stable for the same sources
-    prof = tmp_path / "profiles"
-    prof.mkdir()
+    """A committed DRAM-traffic figure is reported while the files its record
+    names are unchanged, and dropped once one of them changes; files outside
+    the record's list do not matter."""
+    pkg = tmp_path / "hadamard_incoherence_transforms_b200"
+    (pkg / "csrc").mkdir(parents=True)
+    (pkg / "csrc" / "k.cu").write_text("kernel v1")
+    (pkg / "csrc" / "other.cu").write_text("unrelated")
+    (pkg / "build.py").write_text("flags")
+    (tmp_path / "profiles").mkdir()
     monkeypatch.setattr(bench, "ROOT", str(tmp_path))
-    monkeypatch.setattr(bench, "source_digest", lambda: digest)
-    rec = {"k": {"dram_bytes_per_launch": 42.0, "source_digest": digest}}
-    (prof / "traffic.json").write_text(json.dumps(rec))
+    srcs = ["csrc/k.cu", "build.py"]
+    digest = bench.source_digest(srcs)
+    assert len(digest) == 16 and digest == bench.source_digest(srcs)
+    rec = {"k": {"dram_bytes_per_launch": 42.0, "sources": srcs, "source_digest": digest}}
+    (tmp_path / "profiles" / "traffic.json").write_text(json.dumps(rec))
     assert bench.read_profile_traffic("k") == 42.0
     assert bench.read_profile_traffic("other") is None
-    rec["k"]["source_digest"] = "0" * 16
-    (prof / "traffic.json").write_text(json.dumps(rec))
+    (pkg / "csrc" / "other.cu").write_text("changed, but not the kernel's")
+    assert bench.read_profile_traffic("k") == 42.0
+    (pkg / "csrc" / "k.cu").write_text("kernel v2")
     assert bench.read_profile_traffic("k") is None
-    monkeypatch.setattr(bench, "ROOT", real_root)
 
 
 def test_committed_traffic_record_names_the_headline_kernel():
@@ -39,6 +45,10 @@ def test_committed_traffic_record_names_the_headline_kernel():
     assert "k_rows_stream<12,float,float,EPI_QUANT,4>" in rec
     r = rec["k_rows_stream<12,float,float,EPI_QUANT,4>"]
     assert r["dram_bytes_per_launch"] == r["dram_read"] + r["dram_write"]
+    # the record names the kernel's translation unit: k_stream.cu and everything it includes
+    for f in ("csrc/k_stream.cu", "csrc/rows_stream.cuh", "csrc/rows_ops.cuh", "csrc/rows.cuh", "csrc/device.cuh",
+              "csrc/internal.h", "csrc/kernels.h", "build.py"):
+        assert f in r["sources"], f
 
 
 def test_reference_arm_prints_one_contract_line(capsys):
