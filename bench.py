@@ -2,6 +2,7 @@
 
     python bench.py [--gpus N] [--steps K] [--warmup W] [--impl {hit,reference}]
                     [--workload weight_rht_int4|activation_rht|two_sided_lowbit|wht_adapter|two_sided_butterfly]
+                    [--bits 2|3]   (two_sided_lowbit only)
 
 Default workload (the headline metric): fp32 4096 x 4096 weights, row RHT
 (n = 4096, Rademacher signs) fused with symmetric absmax 4-bit RTN in groups
@@ -13,6 +14,9 @@ written once).  Prints one JSON line (rank 0).
 
 --impl reference times the CPU oracle (the reference arm) on a
 bounded sample of the same workload per step.
+
+--gpus N without torchrun re-launches this script under torch.distributed.run
+with N ranks (one per GPU); under torchrun, --gpus must equal WORLD_SIZE.
 """
 from __future__ import annotations
 
@@ -170,7 +174,41 @@ class Workload:
     hot path on rotation set i, host-buffer e2e step, and an oracle sample."""
 
 
-def weight_rht_int4(dev, l2_bytes, host_only=False):
+def _quant_parity(codes_rows, scales_rows, ref, bits, n) -> dict:
+    """Codes and scales of sampled rows against the oracle's: codes differing
+    outside the rounding-boundary window (must be 0), excused ones, and the
+    largest relative scale error."""
+    from oracle import quant as oq
+
+    u = oq.unpack(codes_rows.cpu().numpy(), bits, n)
+    diff = u != ref["u"]
+    win = oq.boundary_window(ref["t"])
+    s = scales_rows.cpu().numpy().astype(np.float64)
+    rs = ref["scales"].astype(np.float64)
+    rel = np.abs(s - rs) / np.where(rs > 0, rs, 1.0)
+    return {"rows": int(u.shape[0]), "codes_outside_window": int((diff & ~win).sum()),
+            "codes_excused": int((diff & win).sum()), "codes": int(u.size),
+            "scale_rel_max": float(rel.max(initial=0.0))}
+
+
+def _rel_l2(got, ref) -> float:
+    ref = np.asarray(ref, np.float64)
+    den = float(np.linalg.norm(ref))
+    return float(np.linalg.norm(np.asarray(got, np.float64) - ref) / (den if den > 0 else 1.0))
+
+
+def _bf16_row_rel(got, ref) -> float:
+    ref = np.asarray(ref, np.float64)
+    d = np.abs(np.asarray(got, np.float64) - ref).max(axis=-1)
+    m = np.abs(ref).max(axis=-1)
+    return float((d / np.where(m > 0, m, 1.0)).max())
+
+
+def _host64(t: torch.Tensor) -> np.ndarray:
+    return t.detach().float().cpu().numpy().astype(np.float64)
+
+
+def weight_rht_int4(dev, l2_bytes, host_only=False, **_):
     import synth
 
     d = synth.weight_rht_int4()
@@ -180,6 +218,7 @@ def weight_rht_int4(dev, l2_bytes, host_only=False):
     w = Workload()
     w.name = "weight_rht_int4"
     w.desc = "fp32 4096x4096 N(0,0.02) + 0.1% outliers x50; row RHT n=4096 + 4-bit absmax RTN g=128, packed"
+    w.io = "fp32 in; 4-bit codes + fp32 scales out"
     w.rows, w.n, w.bytes = rows, n, in_b + out_b
     w.h2d, w.d2h = in_b, out_b
     w.data = d
@@ -192,6 +231,7 @@ def weight_rht_int4(dev, l2_bytes, host_only=False):
 
         q = oq.quantize(oh.rht_rows(d["x"][r0:r1], d["signs"]), bits, group)
         oq.pack(q["u"], bits)
+        return q
 
     w.oracle = oracle
     if host_only:
@@ -211,6 +251,7 @@ def weight_rht_int4(dev, l2_bytes, host_only=False):
         hit.rht_quantize_pack(xs[k], s, bits, group, codes=cs[k], scales=ss[k])
 
     w.step = step
+    w.parity = lambda ref, r0, r1: _quant_parity(cs[0][r0:r1], ss[0][r0:r1], ref, bits, n)
     hx = torch.from_numpy(d["x"]).pin_memory()
     hc = torch.empty(hit.codes_shape(rows, n, bits), dtype=torch.uint8).pin_memory()
     hs = torch.empty((rows, n // group), dtype=torch.float32).pin_memory()
@@ -226,7 +267,7 @@ def weight_rht_int4(dev, l2_bytes, host_only=False):
     return w
 
 
-def activation_rht(dev, l2_bytes, host_only=False):
+def activation_rht(dev, l2_bytes, host_only=False, **_):
     import synth
 
     d = synth.activation_rht()
@@ -234,6 +275,7 @@ def activation_rht(dev, l2_bytes, host_only=False):
     w = Workload()
     w.name, w.rows, w.n = "activation_rht", rows, n
     w.desc = "bf16 8192x4096 0.5*t3 + 1% columns x20; row RHT n=4096, bf16 in/out, fp32 accumulate"
+    w.io = "bf16 in; bf16 out"
     w.bytes = rows * n * 4
     w.h2d = w.d2h = rows * n * 2
     w.kernels_per_step = 1
@@ -242,7 +284,7 @@ def activation_rht(dev, l2_bytes, host_only=False):
     def oracle(r0, r1):
         from oracle import hadamard as oh
 
-        oh.rht_rows(synth.bf16_bits_to_f32(d["x_bf16"][r0:r1]), d["signs"])
+        return oh.rht_rows(synth.bf16_bits_to_f32(d["x_bf16"][r0:r1]), d["signs"])
 
     w.oracle = oracle
     if host_only:
@@ -256,6 +298,7 @@ def activation_rht(dev, l2_bytes, host_only=False):
     s = torch.from_numpy(d["signs"]).to(dev)
     w.rotation = R
     w.step = lambda i: hit.rht_forward(xs[i % R], s, out=ys[i % R])
+    w.parity = lambda ref, r0, r1: {"rows": r1 - r0, "bf16_row_rel_max": _bf16_row_rel(_host64(ys[0][r0:r1]), ref)}
     hx = x0.cpu().pin_memory()
     hy = torch.empty_like(hx).pin_memory()
 
@@ -269,7 +312,7 @@ def activation_rht(dev, l2_bytes, host_only=False):
     return w
 
 
-def two_sided_lowbit(dev, l2_bytes, host_only=False, bits=3):
+def two_sided_lowbit(dev, l2_bytes, host_only=False, bits=3, **_):
     import synth
 
     d = synth.two_sided_lowbit()
@@ -278,19 +321,20 @@ def two_sided_lowbit(dev, l2_bytes, host_only=False, bits=3):
     w = Workload()
     w.name, w.rows, w.n = f"two_sided_lowbit_{bits}b", rows, n
     w.desc = f"bf16 8192x8192 + 0.05% outliers x100; two-sided RHT + {bits}-bit g=64 then dequant + inverse (fp32 out)"
+    w.io = f"bf16 in; {bits}-bit codes + fp32 scales; fp32 reconstruction out"
     q_b = rows * n * bits // 8 + rows * (n // group) * 4
     w.bytes = rows * n * 2 + q_b + q_b + rows * n * 4
     w.h2d, w.d2h = rows * n * 2, rows * n * 4
     w.kernels_per_step = 4  # column pass + row quantize; row dequantize + column pass
     w.kernel_key = "k_cols_cluster<8,bf16,float>"
+    xb = synth.bf16_bits_to_f32(d["x_bf16"])  # the bf16 input widened once (input preparation)
 
     def oracle(r0, r1):
         from oracle import hadamard as oh
         from oracle import quant as oq
 
-        xb = synth.bf16_bits_to_f32(d["x_bf16"])
         idx = np.arange(r0, r1)
-        oq.quantize(oh.two_sided_rows_at(xb, d["row_signs"], d["col_signs"], idx), bits, group)
+        return oq.quantize(oh.two_sided_rows_at(xb, d["row_signs"], d["col_signs"], idx), bits, group)
 
     w.oracle = oracle
     if host_only:
@@ -311,6 +355,21 @@ def two_sided_lowbit(dev, l2_bytes, host_only=False, bits=3):
         hit.dequant_inverse(codes, scales, n, bits, group, rs, col_signs=cs, out=y)
 
     w.step = step
+    w.parity = lambda ref, r0, r1: _quant_parity(codes[r0:r1], scales[r0:r1], ref, bits, n)
+
+    def extra():
+        """Reconstruction MSE of the timed outputs (float64 on the device) next
+        to the oracle's own round-trip MSE (tests/golden, written by the oracle)."""
+        mse = float(((y.double() - x.double()) ** 2).mean().item())
+        try:
+            with open(os.path.join(ROOT, "tests", "golden", "two_sided_lowbit_mse.json")) as f:
+                mse_oracle = float(json.load(f)["mse"][str(bits)])
+        except Exception:
+            mse_oracle = None
+        rel = None if not mse_oracle else abs(mse - mse_oracle) / mse_oracle
+        return {"mse": mse, "mse_oracle": mse_oracle, "mse_rel_diff": rel}
+
+    w.extra = extra
     hx = x.cpu().pin_memory()
     hy = torch.empty((rows, n), dtype=torch.float32).pin_memory()
 
@@ -323,7 +382,7 @@ def two_sided_lowbit(dev, l2_bytes, host_only=False, bits=3):
     return w
 
 
-def wht_adapter(dev, l2_bytes, host_only=False):
+def wht_adapter(dev, l2_bytes, host_only=False, **_):
     import synth
 
     d = synth.wht_adapter()
@@ -331,15 +390,28 @@ def wht_adapter(dev, l2_bytes, host_only=False):
     w = Workload()
     w.name, w.rows, w.n = "wht_adapter", bsz * rows, n
     w.desc = "32 x 4096 x 4096 sparse F (64 nnz/row) -> dense dW = F H/64 (fwd) and grad gather (bwd)"
+    w.io = "fp32 values + int32 columns in; fp32 dense out (fwd); fp32 dense in, fp32 values out (bwd)"
     w.bytes = 2 * (bsz * rows * nnz * 8 + bsz * rows * n * 4)
     w.h2d, w.d2h = bsz * rows * nnz * 8, bsz * rows * nnz * 4
     w.kernels_per_step = 2
     w.kernel_key = "k_rows_b2a<12,float,PRO_SCATTER,0>"
 
     def oracle(r0, r1):
+        # both directions, like the step: expansion of the rows' coefficients,
+        # then the gradient gather from that dense block; flat row r is row
+        # r % rows of matrix r // rows
         from oracle import sparse as osp
 
-        osp.expand(d["values"][:1, r0:r1], d["cols"][:1, r0:r1], n, 1 / 64)
+        dense, grad = [], []
+        r = r0
+        while r < r1:
+            b, a0 = divmod(r, rows)
+            a1 = min(rows, a0 + (r1 - r))
+            dn = osp.expand(d["values"][b:b + 1, a0:a1], d["cols"][b:b + 1, a0:a1], n, 1 / 64)
+            dense.append(dn)
+            grad.append(osp.gather_grad(dn, d["cols"][b:b + 1, a0:a1], 1 / 64))
+            r += a1 - a0
+        return np.concatenate(dense, axis=1), np.concatenate(grad, axis=1)
 
     w.oracle = oracle
     if host_only:
@@ -357,6 +429,8 @@ def wht_adapter(dev, l2_bytes, host_only=False):
         hit.wht_gather(dense, c, 1 / 64, out=g)
 
     w.step = step
+    w.parity = lambda ref, r0, r1: {"rows": r1 - r0, "dense_rel_l2": _rel_l2(_host64(dense[:1, r0:r1]), ref[0]),
+                                    "grad_rel_l2": _rel_l2(_host64(g[:1, r0:r1]), ref[1])}
     hv = v.cpu().pin_memory()
     hg = torch.empty_like(hv).pin_memory()
 
@@ -369,7 +443,7 @@ def wht_adapter(dev, l2_bytes, host_only=False):
     return w
 
 
-def two_sided_butterfly(dev, l2_bytes, host_only=False):
+def two_sided_butterfly(dev, l2_bytes, host_only=False, **_):
     import synth
 
     d = synth.two_sided_butterfly()
@@ -377,6 +451,7 @@ def two_sided_butterfly(dev, l2_bytes, host_only=False):
     w = Workload()
     w.name, w.rows, w.n = "two_sided_butterfly", rows, n
     w.desc = "bf16 4096x14336: R_in (7,16,16,8) along rows then R_out (16,16,16) along columns"
+    w.io = "bf16 in; bf16 out (fp32 between the two sides)"
     w.bytes = rows * n * 4
     w.h2d = w.d2h = rows * n * 2
     w.kernels_per_step = 4  # two row passes (R_in) and two column passes (R_out)
@@ -385,7 +460,7 @@ def two_sided_butterfly(dev, l2_bytes, host_only=False):
     def oracle(r0, r1):
         from oracle import butterfly as ob
 
-        ob.apply_stages(synth.bf16_bits_to_f32(d["x_bf16"][r0:r1]), d["radices_in"], d["blocks_in"])
+        return ob.apply_stages(synth.bf16_bits_to_f32(d["x_bf16"][r0:r1]), d["radices_in"], d["blocks_in"])
 
     w.oracle = oracle
     if host_only:
@@ -404,6 +479,8 @@ def two_sided_butterfly(dev, l2_bytes, host_only=False):
         hit.butterfly_apply(mid, d["radices_out"], bo, axis=0, out=y)
 
     w.step = step
+    # the row side (R_in) of the sampled rows, as held between the two sides
+    w.parity = lambda ref, r0, r1: {"rows": r1 - r0, "row_side_rel_l2": _rel_l2(_host64(mid[r0:r1]), ref)}
     hx = x.cpu().pin_memory()
     hy = torch.empty_like(hx).pin_memory()
 
@@ -457,7 +534,7 @@ def time_oracle(w, budget_s: float, chunk: int) -> tuple[float, int, float]:
 def run_reference(args, world, rank):
     if rank != 0:
         return 0
-    w = WORKLOADS[args.workload](None, 0, host_only=True)
+    w = WORKLOADS[args.workload](None, 0, host_only=True, bits=args.bits)
     per_row = w.bytes / w.rows
     # size one step's sample so warmup + steps finish within about two minutes
     t0 = time.perf_counter()
@@ -509,9 +586,16 @@ def capture_steps(w, steps, first):
 
 
 def time_region(g, stream):
-    """Replay the K-step graph between two events on the launching stream."""
+    """Replay the K-step graph between two events on the launching stream.
+
+    A spin kernel queued ahead of the start event keeps the GPU busy while the
+    host submits the event and the graph, so the timed region starts when the
+    graph's first kernel can start (host submission latency, ~25 us per replay,
+    is not GPU time of the K steps)."""
     start = torch.cuda.Event(enable_timing=True)
     end = torch.cuda.Event(enable_timing=True)
+    with torch.cuda.stream(stream):
+        torch.cuda._sleep(200_000)  # ~0.1 ms at 1.9 GHz, before the start event
     start.record(stream)
     g.replay()
     end.record(stream)
@@ -530,7 +614,7 @@ def run_gpu(args, world, rank, local):
 
     hit.load()  # fails loudly if the extension is missing
     l2 = torch.cuda.get_device_properties(dev).L2_cache_size
-    w = WORKLOADS[args.workload](dev, l2)
+    w = WORKLOADS[args.workload](dev, l2, bits=args.bits)
 
     for i in range(args.warmup):
         w.step(i)
@@ -579,7 +663,7 @@ def run_gpu(args, world, rank, local):
         "metric": METRIC, "value": value, "unit": "GB/s", "n_gpus": world, "steps": args.steps,
         "warmup": args.warmup, "ms_per_step": ms_step, "higher_is_better": True, "scaling": "weak",
         "vs_baseline": None, "dtype": "f32", "data": "synthetic",
-        "config": {"workload": w.desc, "rows": w.rows, "n": w.n,
+        "config": {"workload": w.desc, "io": w.io, "rows": w.rows, "n": w.n,
                    "l2": f"rotating {w.rotation} input/output sets ({w.rotation * w.bytes / 1e6:.0f} MB) vs L2 {l2 / 1e6:.0f} MB",
                    "parallelism": f"replicas x{world}"},
         "rows_per_s": world * w.rows / (ms_step * 1e-3),
@@ -592,17 +676,38 @@ def run_gpu(args, world, rank, local):
         "gpu_launches": args.steps * w.kernels_per_step,
         "clocks": clk.summary(),
     }
+    if hasattr(w, "extra"):
+        line.update(w.extra())
+    # bounded device waits that gave up during the run (0 = every output defined)
+    line["wait_timeouts"] = hit.wait_timeouts()
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         sec, rows_done, rps = time_oracle(w, budget_s=args.cpu_budget, chunk=max(1, min(256, w.rows)))
         line["cpu_baseline"] = {"value": rps * w.bytes / w.rows / 1e9, "unit": "GB/s", "cores": cpu_threads(),
                                 "kind": "oracle",
                                 "sample": f"{rows_done} rows of the {w.rows}-row workload (wrapping) in {sec:.1f} s, scaled to GB/s"}
+        # parity of the timed outputs on the first rows, against the oracle's
+        k = min(8, w.rows)
+        line["cpu_baseline"]["parity"] = w.parity(w.oracle(0, k), 0, k)
     if rank == 0:
         print(json.dumps(line))
     if dist is not None:
         dist.barrier()
         dist.destroy_process_group()
     return 0
+
+
+def relaunch(n: int, argv=None) -> int:
+    """Run this script under torch.distributed.run with n ranks on this node."""
+    import socket
+    import subprocess
+
+    with socket.socket() as sk:
+        sk.bind(("127.0.0.1", 0))
+        port = sk.getsockname()[1]
+    cmd = [sys.executable, "-m", "torch.distributed.run", "--nnodes=1", f"--nproc-per-node={n}",
+           "--master-addr", "127.0.0.1", "--master-port", str(port), os.path.abspath(__file__)]
+    cmd += list(sys.argv[1:] if argv is None else argv)
+    return subprocess.call(cmd)
 
 
 def main(argv=None) -> int:
@@ -614,9 +719,15 @@ def main(argv=None) -> int:
     ap.add_argument("--workload", choices=sorted(WORKLOADS), default="weight_rht_int4")
     ap.add_argument("--cpu-budget", type=float, default=12.0)
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--bits", type=int, choices=[2, 3], default=3, help="code width of two_sided_lowbit")
     args = ap.parse_args(argv)
     args.warmup = max(3, args.warmup)
     world, rank, local = dist_env()
+    if "WORLD_SIZE" not in os.environ and args.gpus > 1:
+        return relaunch(args.gpus, argv)
+    if args.gpus != world:
+        print(json.dumps({"error": f"--gpus {args.gpus} but WORLD_SIZE is {world}"}))
+        return 2
     if args.impl == "reference":
         return run_reference(args, world, rank)
     return run_gpu(args, world, rank, local)

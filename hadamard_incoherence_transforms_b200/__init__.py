@@ -12,6 +12,8 @@ from .api import (  # noqa: F401
     rht_forward,
     rht_inverse,
     rht_quantize_pack,
+    wait_selftest,
+    wait_timeouts,
     wht_expand,
     wht_gather,
     workspace_bytes,

@@ -11,7 +11,7 @@ import os
 
 LIB_PATH = os.path.join(os.path.dirname(os.path.abspath(__file__)), "libhit.so")
 
-HIT_OK, HIT_EINVAL, HIT_EUNSUPPORTED, HIT_EALIGN, HIT_ECUDA, HIT_EWORKSPACE = 0, -1, -2, -3, -4, -5
+HIT_OK, HIT_EINVAL, HIT_EUNSUPPORTED, HIT_EALIGN, HIT_ECUDA, HIT_EWORKSPACE, HIT_ETIMEOUT = 0, -1, -2, -3, -4, -5, -6
 HIT_F32, HIT_BF16 = 0, 1
 HIT_OP_RHT, HIT_OP_QUANT, HIT_OP_DEQUANT, HIT_OP_BUTTERFLY = 0, 1, 2, 3
 
@@ -23,6 +23,8 @@ SIGNATURES = {
     "hit_status_string": (ctypes.c_char_p, [_i32]),
     "hit_last_error": (ctypes.c_char_p, []),
     "hit_workspace_bytes": (_sz, [_i32, _i64, _i64, _i32, _i32]),
+    "hit_wait_timeouts": (_i32, [ctypes.POINTER(ctypes.c_ulonglong), _i32]),
+    "hit_wait_selftest": (_i32, [_i64, _vp]),
     "rht_forward": (_i32, [_vp, _vp, _i64, _i64, _i64, _i64, _i32, _i32, _vp, _i32, _vp, _sz, _vp]),
     "rht_inverse": (_i32, [_vp, _vp, _i64, _i64, _i64, _i64, _i32, _i32, _vp, _i32, _vp, _sz, _vp]),
     "butterfly_apply": (_i32, [_vp, _vp, _i64, _i64, _i64, _i64, _i32, _i32, _i32, _vp, _vp, _vp, _i32, _i32,

@@ -212,3 +212,21 @@ def wht_gather(dense, cols, scale: float, out=None):
     call("wht_expand_sparse", out.data_ptr(), cols.data_ptr(), bsz, rows, n, cols.shape[2], float(scale),
          dense.data_ptr(), 1, _stream(dense.device))
     return out
+
+
+def wait_timeouts(reset: bool = True) -> int:
+    """Bounded device waits that gave up on the current device since the last
+    reset (synchronizes the device).  0 means every output written since then
+    is defined."""
+    n = ctypes.c_ulonglong(0)
+    status = load().hit_wait_timeouts(ctypes.byref(n), int(bool(reset)))
+    if status not in (_lib.HIT_OK, _lib.HIT_ETIMEOUT):
+        raise _lib.HitError("hit_wait_timeouts", status, load().hit_last_error().decode(errors="replace"))
+    return int(n.value)
+
+
+def wait_selftest(limit_ns: int = 1_000_000, device=None) -> None:
+    """Launch one warp whose bounded wait runs out after limit_ns (nothing
+    completes its barrier); wait_timeouts() then counts it."""
+    dev = torch.device("cuda", torch.cuda.current_device()) if device is None else torch.device(device)
+    call("hit_wait_selftest", int(limit_ns), _stream(dev))

@@ -298,11 +298,32 @@ const char* hit_status_string(int status) {
     case HIT_EALIGN: return "misaligned pointer or leading dimension";
     case HIT_ECUDA: return "CUDA error";
     case HIT_EWORKSPACE: return "workspace missing or too small";
+    case HIT_ETIMEOUT: return "a bounded device-side wait gave up";
   }
   return "unknown status";
 }
 
 const char* hit_last_error(void) { return g_last_error.c_str(); }
+
+int hit_wait_timeouts(unsigned long long* count, int reset) {
+  cudaError_t e = cudaDeviceSynchronize();
+  if (e != cudaSuccess) return cuda_status(e, "hit_wait_timeouts: device synchronize");
+  unsigned long long n = 0;
+  e = hit::wait_timeouts_stream(&n, reset != 0);
+  if (e != cudaSuccess) return cuda_status(e, "hit_wait_timeouts: counter read");
+  if (count != nullptr) *count += n;
+  if (n != 0)
+    return fail(HIT_ETIMEOUT, "%llu bounded device wait(s) gave up; outputs written since the last check are undefined",
+                n);
+  return HIT_OK;
+}
+
+int hit_wait_selftest(int64_t limit_ns, void* stream) {
+  if (limit_ns < 1000 || limit_ns > 1000000000)
+    return fail(HIT_EINVAL, "hit_wait_selftest: limit_ns must be in [1000, 1000000000]");
+  return cuda_status(hit::launch_wait_selftest(static_cast<uint64_t>(limit_ns), static_cast<cudaStream_t>(stream)),
+                     "hit_wait_selftest");
+}
 
 size_t hit_workspace_bytes(int op, int64_t rows, int64_t n, int dtype_out, int flags) {
   if (rows <= 0 || n <= 0) return 0;

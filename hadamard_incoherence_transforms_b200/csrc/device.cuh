@@ -238,13 +238,16 @@ __device__ __forceinline__ uint64_t global_ns() {
   asm volatile("mov.u64 %0, %%globaltimer;" : "=l"(t));
   return t;
 }
-// Wait for phase `parity` of an mbarrier; false after about two seconds.
-__device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity) {
+// Time limit of every production wait: far above any legitimate wait (a copy
+// lands in microseconds), short enough that a lost completion ends the kernel.
+constexpr uint64_t kWaitLimitNs = 2000000000ull;
+// Wait for phase `parity` of an mbarrier; false once `limit_ns` has passed.
+__device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, uint64_t limit_ns = kWaitLimitNs) {
   if (mbar_try_wait(bar, parity)) return true;
   const uint64_t t0 = global_ns();
   for (uint32_t i = 1;; ++i) {
     if (mbar_try_wait(bar, parity)) return true;
-    if ((i & 63) == 0 && global_ns() - t0 > 2000000000ull) return false;
+    if ((i & 63) == 0 && global_ns() - t0 > limit_ns) return false;
   }
 }
 // global -> shared bulk copy; dst and src 16-byte aligned, bytes a multiple of 16.

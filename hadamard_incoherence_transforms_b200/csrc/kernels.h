@@ -15,7 +15,10 @@ cudaError_t rows_sparse_all(int logn, int mode, const RowArgs& a, cudaStream_t s
 // Persistent TMA-fed variants for n = 4096 / 8192.
 cudaError_t rows_stream_quant(int logn, int dt_in, int bits, const RowArgs& a, cudaStream_t st);
 cudaError_t rows_stream_store(int logn, int dt_in, int dt_out, const RowArgs& a, cudaStream_t st);
-unsigned int read_wait_timeouts();
+// Bounded-wait timeouts counted on the current device (added to *count; reset
+// clears the counter), and a kernel whose one wait runs out after limit_ns.
+cudaError_t wait_timeouts_stream(unsigned long long* count, bool reset);
+cudaError_t launch_wait_selftest(uint64_t limit_ns, cudaStream_t st);
 // Persistent direct-load variants for n = 4096 / 8192.
 cudaError_t rows_direct_quant(int logn, int dt_in, int bits, const RowArgs& a, cudaStream_t st);
 cudaError_t rows_direct_store(int logn, int dt_in, int dt_out, const RowArgs& a, cudaStream_t st);

@@ -24,7 +24,9 @@ static __device__ __align__(256) float g_noalloc_scratch[kScratchElems];
 
 // Device address of the scratch array, resolved once per device with that
 // device current.  In host code the array's name is only a host-side stand-in,
-// so kernels must be given this address instead.
+// so kernels must be given this address instead.  The address belongs to the
+// device's primary context: a process that destroys that context
+// (cudaDeviceReset) must not call this entry point on the device again.
 constexpr int kMaxDevices = 64;
 std::mutex g_mu;
 void* g_scratch_ptr[kMaxDevices] = {};
@@ -53,8 +55,15 @@ extern "C" HIT_API int rht_quantize_pack_noalloc(const void* x, int64_t rows, in
   if (col_signs == nullptr)  // one-sided: there is no intermediate to place
     return rht_quantize_pack(x, rows, n, ldx, dtype_in, row_signs, nullptr, bits, group, codes, scales, nullptr, 0,
                              stream);
-  if (rows > 0 && n > 0 &&
-      static_cast<unsigned long long>(rows) * static_cast<unsigned long long>(n) > kScratchElems) {
+  // Every argument check of rht_quantize_pack first, with no workspace: that
+  // call launches nothing and answers HIT_EWORKSPACE only when all other
+  // arguments are valid (HIT_OK when there are no rows, else the status a bad
+  // argument gets from rht_quantize_pack itself).
+  const int pre = rht_quantize_pack(x, rows, n, ldx, dtype_in, row_signs, col_signs, bits, group, codes, scales,
+                                    nullptr, 0, stream);
+  if (pre != HIT_EWORKSPACE) return pre;
+  // n is now a power of two in [32, 32768], so the bound cannot overflow.
+  if (rows > static_cast<int64_t>(kScratchElems) / n) {
     hit::set_last_error("rht_quantize_pack_noalloc: rows * n exceeds the static scratch of HIT_NOALLOC_MAX_ELEMS "
                         "(4194304) elements; use rht_quantize_pack with a workspace");
     return HIT_EWORKSPACE;

@@ -67,6 +67,7 @@ extern "C" {
 #define HIT_EALIGN (-3)       /* pointer or leading dimension misaligned */
 #define HIT_ECUDA (-4)        /* a CUDA launch or attribute call failed */
 #define HIT_EWORKSPACE (-5)   /* workspace missing or too small */
+#define HIT_ETIMEOUT (-6)     /* a bounded device-side wait gave up (see hit_wait_timeouts) */
 
 #define HIT_F32 0
 #define HIT_BF16 1
@@ -89,6 +90,30 @@ HIT_API const char* hit_last_error(void);
 /* Bytes of workspace the op needs for a [rows, n] problem with output dtype
  * `dtype_out` (0 means the op needs none).  Workspace must be 16-byte aligned. */
 HIT_API size_t hit_workspace_bytes(int op, int64_t rows, int64_t n, int dtype_out, int flags);
+
+/*
+ * Bounded device-side waits (not an operation of the pages; failure reporting).
+ * The persistent row kernels (row length 4096) wait on shared-memory barriers
+ * for their row copies.  Every such wait is bounded (2 s): one that gives up
+ * stops its warp, leaves that launch's outputs undefined, and increments a
+ * per-device counter instead of hanging the GPU.  Launches cannot report this
+ * through their return value (they are asynchronous), so:
+ *
+ * hit_wait_timeouts: synchronizes the current device (cudaDeviceSynchronize),
+ *   adds the number of waits that gave up on it since the library was loaded
+ *   (or since the last reset) to *count, and clears the counter when `reset`
+ *   is nonzero.  Returns HIT_OK when the count is zero, HIT_ETIMEOUT when it is
+ *   not (every output written since the last check is then suspect), and
+ *   HIT_ECUDA if the device could not be read.  count may be NULL.
+ *
+ * hit_wait_selftest: launches on `stream` one warp that waits, through the
+ *   same bounded-wait routine and counter, on a barrier that nothing ever
+ *   completes, giving up after limit_ns nanoseconds (1000 <= limit_ns <=
+ *   1000000000); a following hit_wait_timeouts then reports it.  Nothing is
+ *   left in flight, so the context stays usable.
+ */
+HIT_API int hit_wait_timeouts(unsigned long long* count, int reset);
+HIT_API int hit_wait_selftest(int64_t limit_ns, void* stream);
 
 /*
  * Randomized Hadamard transform [HARP §1, §2.2; QWHA §2.1].
@@ -202,8 +227,13 @@ HIT_API int wht_expand_sparse(float* values, const int32_t* cols, int64_t batch,
  *    return HIT_EWORKSPACE.  One-sided calls (col_signs == NULL) use no
  *    scratch and have no extra limit.
  *  - The first two-sided call on a device resolves the array's device address
- *    (cudaGetSymbolAddress, with that device current); make that first call
- *    before any stream capture.
+ *    (cudaGetSymbolAddress, with that device current) and keeps it for the
+ *    life of the process; make that first call before any stream capture.  The
+ *    address belongs to the device's primary context: after cudaDeviceReset
+ *    (or anything else that destroys that context) do not call this entry
+ *    point on that device again.
+ *  - Arguments are checked exactly as rht_quantize_pack checks them (same
+ *    statuses) before the size limit below.
  *  - Every call on a device shares the one array and it keeps the last call's
  *    contents (each call overwrites all of the part it reads, so nothing needs
  *    clearing).  Calls whose executions overlap on the GPU -- on different

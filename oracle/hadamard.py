@@ -145,3 +145,16 @@ def rht_rows_chunked(x, signs, chunk: int = 1024) -> np.ndarray:
         cols = np.arange(c0, min(n, c0 + chunk))
         out[..., cols] = rht_rows_at(x, signs, cols)
     return out
+
+
+def irht_rows_chunked(y, signs, chunk: int = 1024) -> np.ndarray:
+    """irht_rows for long rows, building H_n a block of columns at a time:
+    output column j is (y . H[:, j]) / sqrt(n) * s_j (H is symmetric)."""
+    y = np.asarray(y, dtype=np.float64)
+    n = y.shape[-1]
+    s = _signs(signs, n)
+    out = np.empty(y.shape, dtype=np.float64)
+    for c0 in range(0, n, chunk):
+        cols = np.arange(c0, min(n, c0 + chunk))
+        out[..., cols] = (y @ hadamard_rows(n, cols).T) / np.sqrt(n) * s[cols]
+    return out

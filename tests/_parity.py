@@ -1,7 +1,8 @@
 """Comparison helpers for the GPU parity tests (tolerances from the workload
 statement: fp32 transforms within 1e-5 relative L2, bf16 within 2e-2 of each
 row's max |value|, codes bit-exact outside a 1e-6 rounding-boundary window
-with at most 1e-5 of the codes excused, scales within 1e-6 relative)."""
+with at most 1e-5 of the codes excused, scales within 1e-6 relative, and a
+reconstruction MSE within 1e-4 relative of the oracle's own)."""
 import numpy as np
 import torch
 
@@ -12,6 +13,7 @@ F32_REL_L2 = 1e-5
 BF16_ROW_REL = 2e-2
 SCALE_REL = 1e-6
 EXCUSED_FRACTION = 1e-5
+MSE_REL = 1e-4
 
 
 def dev():

@@ -142,3 +142,32 @@ def test_binding_fails_loudly_without_cuda_tensors():
 
     with pytest.raises(ValueError):
         hit.rht_forward(torch.zeros(4, 16))
+
+
+def test_wait_selftest_rejects_limits_on_the_host(lib):
+    # outside [1 us, 1 s]: refused before any launch
+    assert lib.hit_wait_selftest(0, None) == _lib.HIT_EINVAL
+    assert lib.hit_wait_selftest(999, None) == _lib.HIT_EINVAL
+    assert lib.hit_wait_selftest(1_000_000_001, None) == _lib.HIT_EINVAL
+    assert b"timeout" in lib.hit_status_string(_lib.HIT_ETIMEOUT) or b"gave up" in lib.hit_status_string(-6)
+
+
+def test_noalloc_checks_arguments_before_its_size_limit(lib):
+    na = "rht_quantize_pack_noalloc"
+    # a bad n, bits or group with a huge rows * n gets rht_quantize_pack's own status
+    assert status(lib, na, FAKE, 1 << 20, 3000, 3000, 0, None, FAKE, 4, 128, FAKE, FAKE, None) == \
+        _lib.HIT_EUNSUPPORTED
+    assert status(lib, na, FAKE, 1 << 20, 4096, 4096, 0, None, FAKE, 5, 128, FAKE, FAKE, None) == \
+        _lib.HIT_EUNSUPPORTED
+    assert status(lib, na, FAKE, 1 << 20, 4096, 4096, 0, None, FAKE, 4, 100, FAKE, FAKE, None) == \
+        _lib.HIT_EUNSUPPORTED
+    # odd (non power-of-two) rows for a two-sided call
+    assert status(lib, na, FAKE, 3 << 20, 4096, 4096, 0, None, FAKE, 4, 128, FAKE, FAKE, None) == _lib.HIT_EINVAL
+    # rows * n that would wrap around 64 bits is rejected, not wrapped
+    assert status(lib, na, FAKE, 1 << 24, 32768, 32768, 0, None, FAKE, 4, 128, FAKE, FAKE, None) == \
+        _lib.HIT_EWORKSPACE
+    # valid arguments one row above the limit: refused, launching nothing
+    assert status(lib, na, FAKE, 8192, 1024, 1024, 0, None, FAKE, 4, 128, FAKE, FAKE, None) == _lib.HIT_EWORKSPACE
+    assert b"static scratch" in lib.hit_last_error()
+    # no rows: nothing to do
+    assert status(lib, na, FAKE, 0, 1024, 1024, 0, None, FAKE, 4, 128, FAKE, FAKE, None) == _lib.HIT_OK

@@ -8,7 +8,7 @@ import hadamard_incoherence_transforms_b200 as hit
 import synth
 from oracle import hadamard as oh
 from oracle import quant as oq
-from tests._parity import assert_close, check_quant, host, to_gpu_bf16, to_gpu_f32, to_gpu_i8
+from tests._parity import MSE_REL, assert_close, check_quant, host, to_gpu_bf16, to_gpu_f32, to_gpu_i8
 
 pytestmark = pytest.mark.gpu
 
@@ -30,6 +30,11 @@ def test_one_sided_every_length(logn, bits):
     if n > 8192:  # long rows: three rows through the column-blocked oracle
         ref = oq.quantize(oh.rht_rows_chunked(x[:3], s), bits, group)
         check_quant(codes[:3], scales[:3], ref, bits, n)
+        yr = hit.dequant_inverse(codes, scales, n, bits, group, to_gpu_i8(s))
+        torch.cuda.synchronize()
+        u = oq.unpack(codes[:3].cpu().numpy(), bits, n)
+        rec = oh.irht_rows_chunked(oq.dequantize(u, scales[:3].cpu().numpy(), bits, group), s)
+        assert_close(host(yr[:3]), rec, torch.float32, "dequant+inverse (long rows)")
         return
     y64 = oh.rht_rows(x, s)
     ref = oq.quantize(y64, bits, group)
@@ -110,24 +115,28 @@ def test_two_sided_small(rows, n, bits):
 @pytest.mark.parametrize("bits", [2, 3])
 def test_two_sided_lowbit_workload_full_size(bits):
     """bf16 8192 x 8192 with 0.05 % outliers x100, two-sided RHT, groups of 64,
-    then dequant + inverse; 24 sampled rows against the oracle, and the
-    reconstruction MSE of the whole matrix against the oracle's MSE computed on
-    the same sampled rows' exact reconstruction."""
+    then dequant + inverse, at full size: every code and scale against the
+    oracle's; 24 rows of the reconstruction against the oracle's inverse of the
+    GPU's own codes; and the reconstruction MSE of the whole matrix against the
+    MSE of the oracle's own round trip (its codes, its inverse) within 1e-4
+    relative."""
     d = synth.two_sided_lowbit()
     x = to_gpu_bf16(d["x_bf16"])
     rs, cs = to_gpu_i8(d["row_signs"]), to_gpu_i8(d["col_signs"])
     codes, scales = hit.rht_quantize_pack(x, rs, bits, 64, col_signs=cs)
-    torch.cuda.synchronize()
-    xb = synth.bf16_bits_to_f32(d["x_bf16"])
-    rows = np.array([0, 1, 2, 1000, 4095, 4096, 7000, 8191] + list(range(100, 116)))
-    ref = oq.quantize(oh.two_sided_rows_at(xb, d["row_signs"], d["col_signs"], rows), bits, 64)
-    check_quant(codes[rows.tolist()], scales[rows.tolist()], ref, bits, 8192)
     y = hit.dequant_inverse(codes, scales, 8192, bits, 64, rs, col_signs=cs)
     torch.cuda.synchronize()
-    # Reconstruction check: inverse of the GPU's own codes, sampled rows, by the oracle.
+    xb = synth.bf16_bits_to_f32(d["x_bf16"]).astype(np.float64)
+    ref = oq.quantize(oh.two_sided(xb, d["row_signs"], d["col_signs"]), bits, 64)
+    check_quant(codes, scales, ref, bits, 8192)
+    # Reconstruction of the GPU's own codes, sampled rows, by the oracle.
+    rows = np.array([0, 1, 2, 1000, 4095, 4096, 7000, 8191] + list(range(100, 116)))
     u = oq.unpack(codes.cpu().numpy(), bits, 8192)
     yhat = oq.dequantize(u, scales.cpu().numpy(), bits, 64)
     rec_rows = oh.two_sided_inverse_rows_at(yhat, d["row_signs"], d["col_signs"], rows)
     assert_close(host(y[rows.tolist()]), rec_rows, torch.float32, "two-sided reconstruction rows")
-    mse = float(((host(y) - xb) ** 2).mean())
-    assert 0 < mse < float((xb.astype(np.float64) ** 2).mean())
+    # Whole-matrix reconstruction MSE against the oracle's round trip.
+    rec = oh.two_sided_inverse(oq.dequantize(ref["u"], ref["scales"], bits, 64), d["row_signs"], d["col_signs"])
+    mse_oracle = float(((rec - xb) ** 2).mean())
+    mse_gpu = float(((host(y) - xb) ** 2).mean())
+    assert abs(mse_gpu - mse_oracle) <= MSE_REL * mse_oracle, f"MSE {mse_gpu:.9e} vs oracle {mse_oracle:.9e}"

@@ -122,3 +122,19 @@ def test_sampled_inverse_and_chunked_forward():
     np.testing.assert_allclose(oh.two_sided_inverse_rows_at(wp, s_in, s_out, rows),
                                oh.two_sided_inverse(wp, s_in, s_out)[rows], atol=1e-12)
     np.testing.assert_allclose(oh.rht_rows_chunked(wp, s_in, chunk=48), oh.rht_rows(wp, s_in), atol=1e-12)
+    np.testing.assert_allclose(oh.irht_rows_chunked(wp, s_in, chunk=48), oh.irht_rows(wp, s_in), atol=1e-12)
+
+
+def test_chunked_inverse_undoes_chunked_forward():
+    # signs after H on the inverse side: a sign error or a missing 1/sqrt(n)
+    # breaks the round trip on rows long enough to need the chunked forms
+    rng = np.random.default_rng(23)
+    n = 4096
+    x = rng.standard_normal((2, n))
+    s = rng.choice([-1, 1], n)
+    back = oh.irht_rows_chunked(oh.rht_rows_chunked(x, s, chunk=1000), s, chunk=777)
+    np.testing.assert_allclose(back, x, atol=1e-10)
+    # e_0 through the inverse is s * (first column of H) / sqrt(n)
+    e0 = np.zeros((1, n))
+    e0[0, 0] = 1.0
+    np.testing.assert_allclose(oh.irht_rows_chunked(e0, s, chunk=999)[0], s / np.sqrt(n), atol=1e-15)
