@@ -22,6 +22,9 @@ Readings taken where the pages stop:
   set to n and the rest re-split, until none passes; the shares are rounded
   down and the units left over go one each to the largest fractional parts
   (ties to the lower row).  If every uncapped e_r is zero the split is equal.
+  The share of row r is (R' * e_r) / S in float64, with R' the units left for
+  the uncapped rows and S the sum of their errors taken left to right in
+  float64 (a fixed order, so any implementation can reproduce the split).
 * Selection inside a row: the k_r largest |F*_{r,j}|, ties to the lower j; the
   chosen columns are returned in ascending order.
 * Direct values: c = F*[r, E_r].  Refined values: per row, the least-squares
@@ -72,6 +75,14 @@ def channel_error(dw, x=None) -> np.ndarray:
     return np.sqrt(np.sum(out * out, axis=-1))
 
 
+def _sum_left_to_right(v) -> float:
+    """sum(v) in float64, one element after the other from the first."""
+    acc = 0.0
+    for x in np.asarray(v, dtype=np.float64).tolist():
+        acc += x
+    return acc
+
+
 def allocate(err, budget: int, k_min: int, n: int) -> np.ndarray:
     """Per-row counts k_r (int64) summing to budget, each in [k_min, n]."""
     e = np.asarray(err, dtype=np.float64)
@@ -85,9 +96,10 @@ def allocate(err, budget: int, k_min: int, n: int) -> np.ndarray:
         free = ~capped
         rest = left - room * int(capped.sum())
         w = e[free]
-        w = w if w.sum() > 0 else np.ones_like(w)
+        if _sum_left_to_right(w) <= 0:
+            w = np.ones_like(w)
         share = np.zeros(rows)
-        share[free] = rest * w / w.sum()
+        share[free] = (float(rest) * w) / _sum_left_to_right(w)
         over = free & (share > room)
         if not over.any():
             break
