@@ -1,7 +1,8 @@
 """Benchmark of the fused RHT + group-quantization hot path on B200.
 
     python bench.py [--gpus N] [--steps K] [--warmup W] [--impl {hit,reference}]
-                    [--workload weight_rht_int4|activation_rht|two_sided_lowbit|wht_adapter|two_sided_butterfly]
+                    [--workload weight_rht_int4|activation_rht|activation_quant|two_sided_lowbit|wht_adapter|
+                                two_sided_butterfly|mixed_rht_int4|harp_rotation]
                     [--bits 2|3]   (two_sided_lowbit only)
 
 Default workload (the headline metric): fp32 4096 x 4096 weights, row RHT
@@ -312,6 +313,65 @@ def activation_rht(dev, l2_bytes, host_only=False, **_):
     return w
 
 
+def activation_quant(dev, l2_bytes, host_only=False, **_):
+    import synth
+
+    d = synth.activation_rht()
+    rows, n, bits, group = 8192, 4096, 4, 4096
+    w = Workload()
+    w.name, w.rows, w.n = "activation_quant", rows, n
+    w.desc = "bf16 8192x4096 0.5*t3 + 1% columns x20; row RHT n=4096 + 4-bit absmax RTN, one scale per token"
+    w.io = "bf16 in; 4-bit codes + fp32 per-token scales out"
+    in_b = rows * n * 2
+    out_b = rows * n * bits // 8 + rows * 4
+    w.bytes = in_b + out_b
+    w.h2d, w.d2h = in_b, out_b
+    w.kernels_per_step = 1
+    w.kernel_key = "k_rows_stream<12,bf16,float,EPI_QUANT,4>"
+    xb = synth.bf16_bits_to_f32(d["x_bf16"])
+
+    def oracle(r0, r1):
+        from oracle import hadamard as oh
+        from oracle import quant as oq
+
+        q = oq.quantize(oh.rht_rows(xb[r0:r1], d["signs"]), bits, group)
+        oq.pack(q["u"], bits)
+        return q
+
+    w.oracle = oracle
+    if host_only:
+        return w
+    import hadamard_incoherence_transforms_b200 as hit
+
+    R = max(2, math.ceil(4 * l2_bytes / w.bytes) + 1)
+    x0 = torch.from_numpy(d["x_bf16"].view(np.int16)).to(dev).view(torch.bfloat16)
+    xs = [x0] + [x0.clone() for _ in range(R - 1)]
+    s = torch.from_numpy(d["signs"]).to(dev)
+    cs = [torch.empty(hit.codes_shape(rows, n, bits), dtype=torch.uint8, device=dev) for _ in range(R)]
+    ss = [torch.empty((rows, 1), dtype=torch.float32, device=dev) for _ in range(R)]
+    w.rotation = R
+
+    def step(i):
+        k = i % R
+        hit.rht_quantize_pack(xs[k], s, bits, group, codes=cs[k], scales=ss[k])
+
+    w.step = step
+    w.parity = lambda ref, r0, r1: _quant_parity(cs[0][r0:r1], ss[0][r0:r1], ref, bits, n)
+    hx = x0.cpu().pin_memory()
+    hc = torch.empty(hit.codes_shape(rows, n, bits), dtype=torch.uint8).pin_memory()
+    hs = torch.empty((rows, 1), dtype=torch.float32).pin_memory()
+
+    def e2e_step(i):
+        k = i % R
+        xs[k].copy_(hx, non_blocking=True)
+        hit.rht_quantize_pack(xs[k], s, bits, group, codes=cs[k], scales=ss[k])
+        hc.copy_(cs[k], non_blocking=True)
+        hs.copy_(ss[k], non_blocking=True)
+
+    w.e2e_step = e2e_step
+    return w
+
+
 def two_sided_lowbit(dev, l2_bytes, host_only=False, bits=3, **_):
     import synth
 
@@ -493,12 +553,128 @@ def two_sided_butterfly(dev, l2_bytes, host_only=False, **_):
     return w
 
 
+def mixed_rht_int4(dev, l2_bytes, host_only=False, **_):
+    import synth
+
+    d = synth.mixed_rht_int4()
+    rows, n, bits, group = 4096, 5120, 4, 128
+    w = Workload()
+    w.name, w.rows, w.n = "mixed_rht_int4", rows, n
+    w.desc = ("fp32 4096x5120 N(0,0.02) + 0.1% outliers x50; mixed-radix RHT (8,8,8,5,2), QR mixer for radix 5, "
+              "+ 4-bit absmax RTN g=128, packed")
+    w.io = "fp32 in; 4-bit codes + fp32 scales out"
+    in_b = rows * n * 4
+    out_b = rows * n * bits // 8 + rows * (n // group) * 4
+    w.bytes = in_b + out_b
+    w.h2d, w.d2h = in_b, out_b
+    w.kernels_per_step = 1
+    w.kernel_key = "k_rows_mixed5120_q4"
+    g5 = d["mixers"][5][0]
+
+    def oracle(r0, r1):
+        from oracle import butterfly as ob
+        from oracle import quant as oq
+
+        blocks = ob.rht_stage_blocks(d["radices"], d["mixers"])
+        q = oq.quantize(ob.rht_mixed(d["x"][r0:r1], d["signs"], d["radices"], blocks), bits, group)
+        oq.pack(q["u"], bits)
+        return q
+
+    w.oracle = oracle
+    if host_only:
+        return w
+    import hadamard_incoherence_transforms_b200 as hit
+
+    R = max(2, math.ceil(4 * l2_bytes / w.bytes) + 1)
+    x0 = torch.from_numpy(d["x"]).to(dev)
+    xs = [x0] + [x0.clone() for _ in range(R - 1)]
+    s = torch.from_numpy(d["signs"]).to(dev)
+    cs = [torch.empty(hit.codes_shape(rows, n, bits), dtype=torch.uint8, device=dev) for _ in range(R)]
+    ss = [torch.empty((rows, n // group), dtype=torch.float32, device=dev) for _ in range(R)]
+    w.rotation = R
+
+    def step(i):
+        k = i % R
+        hit.rht_mixed_quantize_pack(xs[k], s, g5, codes=cs[k], scales=ss[k])
+
+    w.step = step
+    w.parity = lambda ref, r0, r1: _quant_parity(cs[0][r0:r1], ss[0][r0:r1], ref, bits, n)
+    hx = torch.from_numpy(d["x"]).pin_memory()
+    hc = torch.empty(hit.codes_shape(rows, n, bits), dtype=torch.uint8).pin_memory()
+    hs = torch.empty((rows, n // group), dtype=torch.float32).pin_memory()
+
+    def e2e_step(i):
+        k = i % R
+        xs[k].copy_(hx, non_blocking=True)
+        hit.rht_mixed_quantize_pack(xs[k], s, g5, codes=cs[k], scales=ss[k])
+        hc.copy_(cs[k], non_blocking=True)
+        hs.copy_(ss[k], non_blocking=True)
+
+    w.e2e_step = e2e_step
+    return w
+
+
+def harp_rotation(dev, l2_bytes, host_only=False, **_):
+    import synth
+
+    d = synth.harp_rotation()
+    rows, n = 4096, 4096
+    radices = d["radices"]
+    w = Workload()
+    w.name, w.rows, w.n = "harp_rotation", rows, n
+    w.desc = ("fp32 4096x4096 weights; HARP blocks Q(theta) G_16 built on the device for radices (16,16,16) "
+              "(Cayley, theta ~ N(0,0.05)), signs folded into stage 0, then y = R(theta) diag(s) x")
+    w.io = "fp32 in; fp32 out"
+    w.bytes = rows * n * 8
+    w.h2d = w.d2h = rows * n * 4
+    w.kernels_per_step = 3 + 2  # three block builds, two butterfly passes
+    w.kernel_key = "k_bfly_pass"
+
+    def oracle(r0, r1):
+        from oracle import harp as oha
+
+        return oha.forward(d["x"][r0:r1], d["signs"], radices, d["thetas"], d["base_mixers"])
+
+    w.oracle = oracle
+    if host_only:
+        return w
+    import hadamard_incoherence_transforms_b200 as hit
+
+    x = torch.from_numpy(d["x"]).to(dev)
+    s = torch.from_numpy(d["signs"]).to(dev)
+    th = [torch.from_numpy(t).to(dev) for t in d["thetas"]]
+    blocks = [torch.empty((n // b, b, b), dtype=torch.float32, device=dev) for b in radices]
+    y = torch.empty_like(x)
+    w.rotation = 1
+
+    def step(i):
+        for t, b in enumerate(radices):
+            hit.harp_blocks(th[t], b, signs=s if t == 0 else None, out=blocks[t])
+        hit.butterfly_apply(x, radices, blocks, out=y)
+
+    w.step = step
+    w.parity = lambda ref, r0, r1: {"rows": r1 - r0, "rel_l2": _rel_l2(_host64(y[r0:r1]), ref)}
+    hx = x.cpu().pin_memory()
+    hy = torch.empty_like(hx).pin_memory()
+
+    def e2e_step(i):
+        x.copy_(hx, non_blocking=True)
+        step(i)
+        hy.copy_(y, non_blocking=True)
+
+    w.e2e_step = e2e_step
+    return w
+
+
 WORKLOADS = {
     "weight_rht_int4": weight_rht_int4,
+    "activation_quant": activation_quant,
     "activation_rht": activation_rht,
     "two_sided_lowbit": two_sided_lowbit,
     "wht_adapter": wht_adapter,
     "two_sided_butterfly": two_sided_butterfly,
+    "mixed_rht_int4": mixed_rht_int4,
+    "harp_rotation": harp_rotation,
 }
 
 

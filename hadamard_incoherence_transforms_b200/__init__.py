@@ -9,13 +9,21 @@ from .api import (  # noqa: F401
     butterfly_apply,
     codes_shape,
     dequant_inverse,
+    harp_blocks,
+    harp_n_params,
+    qwha_allocate,
+    qwha_select,
     rht_forward,
     rht_inverse,
+    rht_mixed_quantize_pack,
     rht_quantize_pack,
+    row_norms,
     wait_selftest,
     wait_timeouts,
     wht_expand,
+    wht_expand_2d,
     wht_gather,
+    wht_gather_2d,
     workspace_bytes,
 )
 

@@ -30,8 +30,14 @@ SIGNATURES = {
     "butterfly_apply": (_i32, [_vp, _vp, _i64, _i64, _i64, _i64, _i32, _i32, _i32, _vp, _vp, _vp, _i32, _i32,
                                _vp, _sz, _vp]),
     "rht_quantize_pack": (_i32, [_vp, _i64, _i64, _i64, _i32, _vp, _vp, _i32, _i32, _vp, _vp, _vp, _sz, _vp]),
+    "rht_mixed_quantize_pack": (_i32, [_vp, _i64, _i64, _i64, _vp, _vp, _i32, _i32, _vp, _vp, _vp]),
     "dequant_inverse": (_i32, [_vp, _vp, _i64, _i64, _i32, _i32, _vp, _vp, _vp, _i64, _i32, _vp, _sz, _vp]),
     "wht_expand_sparse": (_i32, [_vp, _vp, _i64, _i64, _i64, _i32, ctypes.c_float, _vp, _i32, _vp]),
+    "wht_expand_sparse_2d": (_i32, [_vp, _vp, _i64, _i64, _i64, _i32, ctypes.c_float, _vp, _i32, _vp, _sz, _vp]),
+    "row_norms": (_i32, [_vp, _i64, _i64, _i64, _vp, _vp]),
+    "qwha_allocate": (_i32, [_vp, _i64, _i64, _i64, _i64, _vp]),
+    "qwha_select": (_i32, [_vp, _i64, _i64, _i64, _vp, _vp, _vp, _vp]),
+    "harp_blocks": (_i32, [_vp, _vp, ctypes.c_float, _i64, _i32, _vp, _vp, _vp, _vp]),
     "rht_quantize_pack_noalloc": (_i32, [_vp, _i64, _i64, _i64, _i32, _vp, _vp, _i32, _i32, _vp, _vp, _vp]),
 }
 

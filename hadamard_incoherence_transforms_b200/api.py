@@ -230,3 +230,137 @@ def wait_selftest(limit_ns: int = 1_000_000, device=None) -> None:
     completes its barrier); wait_timeouts() then counts it."""
     dev = torch.device("cuda", torch.cuda.current_device()) if device is None else torch.device(device)
     call("hit_wait_selftest", int(limit_ns), _stream(dev))
+
+
+def harp_n_params(b: int) -> int:
+    """Learnable parameters per b x b HARP block: 0 (b = 1), 1 (b = 2), b(b-1)/2."""
+    return 0 if b == 1 else 1 if b == 2 else b * (b - 1) // 2
+
+
+def harp_blocks(theta, b: int, mixer=None, signs=None, theta_scale: float | None = None, groups: int | None = None,
+                out=None):
+    """Blocks [groups, b, b] of one HARP stage, B_c = Q(theta_c) G_b.
+
+    theta: float32 [groups, P] or int8 [groups, P] (then theta_scale is the
+    per-stage scale of the stored parameters); None for b = 1 (give groups).
+    mixer: float32 [b, b] (None = Sylvester / sqrt(b) for powers of two).
+    signs: int8 [b * groups] to fold the RHT sign vector into a first stage."""
+    if theta is not None:
+        _cuda(theta, "theta")
+        if theta.dim() != 2 or theta.shape[1] != harp_n_params(b) or not theta.is_contiguous():
+            raise ValueError(f"theta must be contiguous [groups, {harp_n_params(b)}]")
+        groups = theta.shape[0]
+        if theta.dtype == torch.int8:
+            if theta_scale is None:
+                raise ValueError("int8 theta needs theta_scale")
+        elif theta.dtype != torch.float32:
+            raise ValueError("theta must be float32 or int8")
+    elif groups is None:
+        raise ValueError("give theta or groups")
+    dev = theta.device if theta is not None else torch.device("cuda", torch.cuda.current_device())
+    if mixer is not None:
+        _cuda(mixer, "mixer")
+        if mixer.shape != (b, b) or mixer.dtype != torch.float32 or not mixer.is_contiguous():
+            raise ValueError(f"mixer must be contiguous float32 [{b}, {b}]")
+    if signs is not None:
+        _cuda(signs, "signs")
+        if signs.dtype != torch.int8 or signs.numel() != b * groups or not signs.is_contiguous():
+            raise ValueError(f"signs must be contiguous int8 of length {b * groups}")
+    if out is None:
+        out = torch.empty((groups, b, b), dtype=torch.float32, device=dev)
+    q = theta is not None and theta.dtype == torch.int8
+    call("harp_blocks", None if q or theta is None else theta.data_ptr(), theta.data_ptr() if q else None,
+         float(theta_scale or 1.0), groups, b, _ptr(mixer), _ptr(signs), out.data_ptr(), _stream(dev))
+    return out
+
+
+def rht_mixed_quantize_pack(x, signs, mixer5, bits: int = 4, group: int = 128, codes=None, scales=None):
+    """d = 5120 rows: y = R diag(s) x with the schedule (8, 8, 8, 5, 2) (Hadamard
+    blocks for the power-of-two radices, the given 5 x 5 orthogonal mixer for
+    radix 5), then 4-bit absmax RTN in groups of 128.  Returns (codes, scales)."""
+    x = _mat(x, "x")
+    rows, n = x.shape
+    if x.dtype != torch.float32:
+        raise ValueError("x must be float32")
+    g = [float(v) for v in (mixer5.flatten().tolist() if hasattr(mixer5, "flatten") else mixer5)]
+    if len(g) != 25:
+        raise ValueError("mixer5 must have 25 entries (5 x 5, row-major)")
+    gh = (ctypes.c_float * 25)(*g)
+    if codes is None:
+        codes = torch.empty(codes_shape(rows, n, bits), dtype=torch.uint8, device=x.device)
+    if scales is None:
+        scales = torch.empty((rows, n // group), dtype=torch.float32, device=x.device)
+    s = _signs(signs, n, "signs")
+    call("rht_mixed_quantize_pack", x.data_ptr(), rows, n, x.stride(0), _ptr(s), ctypes.cast(gh, ctypes.c_void_p),
+         bits, group, codes.data_ptr(), scales.data_ptr(), _stream(x.device))
+    return codes, scales
+
+
+def wht_expand_2d(values, cols, n: int, scale: float, out=None):
+    """dense[b] = (H_m / sqrt m) scatter(values, cols)[b] H_n * scale, m = values.shape[1]."""
+    _sparse_check(values, cols)
+    bsz, m, nnz = values.shape
+    if out is None:
+        out = torch.empty((bsz, m, n), dtype=torch.float32, device=values.device)
+    _cuda(out, "out")
+    if out.shape != (bsz, m, n) or out.dtype != torch.float32 or not out.is_contiguous():
+        raise ValueError("out must be contiguous float32 [batch, m, n]")
+    call("wht_expand_sparse_2d", values.data_ptr(), cols.data_ptr(), bsz, m, n, nnz, float(scale), out.data_ptr(), 0,
+         None, 0, _stream(values.device))
+    return out
+
+
+def wht_gather_2d(dense, cols, scale: float, out=None, workspace=None):
+    """values[b, r, k] = ((H_m / sqrt m) dense[b] H_n * scale)[r, cols[b, r, k]] (the gradient of wht_expand_2d)."""
+    _cuda(dense, "dense")
+    bsz, m, n = dense.shape
+    if dense.dtype != torch.float32 or not dense.is_contiguous():
+        raise ValueError("dense must be contiguous float32 [batch, m, n]")
+    if out is None:
+        out = torch.empty(cols.shape, dtype=torch.float32, device=dense.device)
+    _sparse_check(out, cols)
+    ws = workspace if workspace is not None else torch.empty(bsz * m * n, dtype=torch.float32, device=dense.device)
+    call("wht_expand_sparse_2d", out.data_ptr(), cols.data_ptr(), bsz, m, n, cols.shape[2], float(scale),
+         dense.data_ptr(), 1, ws.data_ptr(), ws.numel() * ws.element_size(), _stream(dense.device))
+    return out
+
+
+def row_norms(x, out=None):
+    """||x_r||_2 per row of an fp32 matrix, accumulated in fp64 (float64 [rows])."""
+    x = _mat(x, "x")
+    rows, n = x.shape
+    if x.dtype != torch.float32:
+        raise ValueError("x must be float32")
+    if out is None:
+        out = torch.empty(rows, dtype=torch.float64, device=x.device)
+    call("row_norms", x.data_ptr(), rows, n, x.stride(0), out.data_ptr(), _stream(x.device))
+    return out
+
+
+def qwha_allocate(err, budget: int, k_min: int, n: int):
+    """AdaAlloc budget split (host arithmetic): int64 numpy counts per row."""
+    import numpy as np
+
+    e = np.ascontiguousarray(np.asarray(err, dtype=np.float64))
+    counts = np.zeros(e.shape[0], dtype=np.int64)
+    call("qwha_allocate", e.ctypes.data_as(ctypes.c_void_p), e.shape[0], int(budget), int(k_min), int(n),
+         counts.ctypes.data_as(ctypes.c_void_p))
+    return counts
+
+
+def qwha_select(f, offsets, cols=None, values=None):
+    """Per-row top-|f| selection on the device (CSR offsets int64 [rows + 1] on the
+    device); returns (cols int32, values float32) in ascending column order per row."""
+    f = _mat(f, "f")
+    rows, n = f.shape
+    _cuda(offsets, "offsets")
+    if offsets.dtype != torch.int64 or offsets.numel() != rows + 1 or not offsets.is_contiguous():
+        raise ValueError("offsets must be contiguous int64 [rows + 1]")
+    total = int(offsets[-1].item())
+    if cols is None:
+        cols = torch.empty(total, dtype=torch.int32, device=f.device)
+    if values is None:
+        values = torch.empty(total, dtype=torch.float32, device=f.device)
+    call("qwha_select", f.data_ptr(), rows, n, f.stride(0), offsets.data_ptr(), cols.data_ptr(), values.data_ptr(),
+         _stream(f.device))
+    return cols, values

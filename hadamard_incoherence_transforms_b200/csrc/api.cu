@@ -310,6 +310,7 @@ int hit_wait_timeouts(unsigned long long* count, int reset) {
   if (e != cudaSuccess) return cuda_status(e, "hit_wait_timeouts: device synchronize");
   unsigned long long n = 0;
   e = hit::wait_timeouts_stream(&n, reset != 0);
+  if (e == cudaSuccess) e = hit::wait_timeouts_mixed(&n, reset != 0);
   if (e != cudaSuccess) return cuda_status(e, "hit_wait_timeouts: counter read");
   if (count != nullptr) *count += n;
   if (n != 0)
@@ -506,6 +507,26 @@ int rht_quantize_pack(const void* x, int64_t rows, int64_t n, int64_t ldx, int d
   return cuda_status(e, fn);
 }
 
+int rht_mixed_quantize_pack(const float* x, int64_t rows, int64_t n, int64_t ldx, const int8_t* signs,
+                            const float* mixer, int bits, int group, uint8_t* codes, float* scales, void* stream) {
+  const char* fn = "rht_mixed_quantize_pack";
+  if (rows < 0) return fail(HIT_EINVAL, "%s: rows < 0", fn);
+  if (n != 5120) return fail(HIT_EUNSUPPORTED, "%s: n must be 5120 (radices 8, 8, 8, 5, 2)", fn);
+  if (bits != 4 || group != 128) return fail(HIT_EUNSUPPORTED, "%s: 4-bit codes in groups of 128 only", fn);
+  if (mixer == nullptr) return fail(HIT_EINVAL, "%s: the 5 x 5 mixer is required", fn);
+  if (rows == 0) return ok();
+  if (x == nullptr || codes == nullptr || scales == nullptr) return fail(HIT_EINVAL, "%s: NULL operand", fn);
+  if (ldx < n) return fail(HIT_EINVAL, "%s: leading dimension %lld < n", fn, (long long)ldx);
+  if (!aligned(x, 16) || ldx % 4 != 0) return fail(HIT_EALIGN, "%s: x and its row pitch must be 16-byte aligned", fn);
+  if (!aligned(codes, 16) || !aligned(scales, 4))
+    return fail(HIT_EALIGN, "%s: codes must be 16-byte, scales 4-byte aligned", fn);
+  for (int i = 0; i < 25; ++i)
+    if (!std::isfinite(mixer[i])) return fail(HIT_EINVAL, "%s: mixer entries must be finite", fn);
+  return cuda_status(hit::rows_mixed5120_quant(x, rows, ldx, signs, mixer, codes, scales,
+                                               static_cast<cudaStream_t>(stream)),
+                     fn);
+}
+
 int dequant_inverse(const uint8_t* codes, const float* scales, int64_t rows, int64_t n, int bits, int group,
                     const int8_t* row_signs, const int8_t* col_signs, void* y, int64_t ldy, int dtype_out,
                     void* workspace, size_t workspace_bytes, void* stream) {
@@ -592,6 +613,60 @@ int wht_expand_sparse(float* values, const int32_t* cols, int64_t batch, int64_t
     a.sp_out = values;
   }
   return cuda_status(hit::rows_sparse_all(ilog2(n), mode, a, static_cast<cudaStream_t>(stream)), fn);
+}
+
+int wht_expand_sparse_2d(float* values, const int32_t* cols, int64_t batch, int64_t m, int64_t n, int32_t nnz,
+                         float scale, float* dense, int mode, void* workspace, size_t workspace_bytes, void* stream) {
+  const char* fn = "wht_expand_sparse_2d";
+  if (batch < 0 || m < 1) return fail(HIT_EINVAL, "%s: bad batch or m", fn);
+  if (!is_pow2(m) || m > (int64_t(1) << 24)) return fail(HIT_EUNSUPPORTED, "%s: m must be a power of two <= 2^24", fn);
+  if (!is_pow2(n) || n < 32 || n > 32768) return fail(HIT_EUNSUPPORTED, "%s: n must be a power of two in [32, 32768]", fn);
+  if (nnz < 1 || nnz > n) return fail(HIT_EINVAL, "%s: nnz must be in [1, n]", fn);
+  if (mode != 0 && mode != 1) return fail(HIT_EINVAL, "%s: mode must be 0 or 1", fn);
+  if (batch == 0) return ok();
+  if (values == nullptr || cols == nullptr || dense == nullptr) return fail(HIT_EINVAL, "%s: NULL operand", fn);
+  if (!aligned(values, 4) || !aligned(cols, 4) || !aligned(dense, 16)) return fail(HIT_EALIGN, "%s: misaligned operand", fn);
+  const size_t mat = static_cast<size_t>(m) * static_cast<size_t>(n);
+  float* g = nullptr;
+  if (mode == 1) {
+    const size_t need = static_cast<size_t>(batch) * mat * 4;
+    if (workspace == nullptr || workspace_bytes < need) return fail(HIT_EWORKSPACE, "%s: needs %zu workspace bytes", fn, need);
+    if (!aligned(workspace, 16)) return fail(HIT_EALIGN, "%s: workspace must be 16-byte aligned", fn);
+    g = static_cast<float*>(workspace);
+  }
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  hit::RowArgs a;
+  a.rows = batch * m;
+  a.nnz = nnz;
+  a.sp_cols = cols;
+  a.sp_scale = scale;
+  if (mode == 0) {
+    // rows: scatter + transform (times scale) into dense; then every column
+    // of every matrix in place (orthonormal, 1/sqrt(m))
+    a.sp_values = values;
+    a.y = dense;
+    a.ldy = n;
+    int r = cuda_status(hit::rows_sparse_all(ilog2(n), 0, a, st), fn);
+    if (r) return r;
+    for (int64_t b = 0; b < batch; ++b) {
+      float* d = dense + static_cast<size_t>(b) * mat;
+      r = run_cols(d, HIT_F32, n, d, HIT_F32, n, m, n, nullptr, nullptr, d, n, st);
+      if (r) return r;
+    }
+    return HIT_OK;
+  }
+  // gradient: columns of every matrix of the incoming dense gradient into the
+  // workspace, then rows: transform (times scale) + gather
+  for (int64_t b = 0; b < batch; ++b) {
+    float* d = dense + static_cast<size_t>(b) * mat;
+    float* w = g + static_cast<size_t>(b) * mat;
+    const int r = run_cols(d, HIT_F32, n, w, HIT_F32, n, m, n, nullptr, nullptr, w, n, st);
+    if (r) return r;
+  }
+  a.x = g;
+  a.ldx = n;
+  a.sp_out = values;
+  return cuda_status(hit::rows_sparse_all(ilog2(n), 1, a, st), fn);
 }
 
 }  // extern "C"

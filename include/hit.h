@@ -93,7 +93,7 @@ HIT_API size_t hit_workspace_bytes(int op, int64_t rows, int64_t n, int dtype_ou
 
 /*
  * Bounded device-side waits (not an operation of the pages; failure reporting).
- * The persistent row kernels (row length 4096) wait on shared-memory barriers
+ * The persistent row kernels (row lengths 4096 and 5120) wait on shared-memory barriers
  * for their row copies.  Every such wait is bounded (2 s): one that gives up
  * stops its warp, leaves that launch's outputs undefined, and increments a
  * per-device counter instead of hanging the GPU.  Launches cannot report this
@@ -183,6 +183,26 @@ HIT_API int rht_quantize_pack(const void* x, int64_t rows, int64_t n, int64_t ld
                       void* stream);
 
 /*
+ * Fused randomized transform of the non-power-of-two length n = 5120 + group
+ * quantization [HARP §2.1: mixed-radix schedules such as (8, 8, 8, 5, 2) for
+ * d = 5120, with an orthogonal mixer (QR of a Gaussian) for the radix that is
+ * not a power of two; §2.2: the mixers of power-of-two radices are the
+ * normalized Sylvester Hadamard blocks].
+ * Each row is transformed by y = R diag(signs) x with R the stage product of
+ * the schedule (8, 8, 8, 5, 2) (the butterfly_apply digit convention) whose
+ * radix-8 and radix-2 blocks are H_b / sqrt(b) and whose radix-5 blocks are
+ * all the given mixer G_5; equivalently R = (H_512 / sqrt 512) (x) G_5 (x)
+ * (H_2 / sqrt 2).  Then 4-bit symmetric absmax RTN in groups of 128 exactly as
+ * rht_quantize_pack: codes uint8 [rows, 2560], scales fp32 [rows, 40].
+ * x: fp32 [rows, ldx], 16-byte aligned rows.  signs: int8 [5120] or NULL.
+ * mixer: HOST pointer to the 25 fp32 entries of G_5 (row-major, orthogonal).
+ * n must be 5120, bits 4 and group 128 (HIT_EUNSUPPORTED otherwise).
+ */
+HIT_API int rht_mixed_quantize_pack(const float* x, int64_t rows, int64_t n, int64_t ldx, const int8_t* signs,
+                                    const float* mixer, int bits, int group, uint8_t* codes, float* scales,
+                                    void* stream);
+
+/*
  * Dequantize then inverse-transform [HARP §5: exact change of basis, so the
  * reconstruction is the inverse rotation of the dequantized codes].
  * codes / scales as written by rht_quantize_pack; yhat = fp32(u - 2^(bits-1)) * s.
@@ -210,6 +230,84 @@ HIT_API int dequant_inverse(const uint8_t* codes, const float* scales, int64_t r
  */
 HIT_API int wht_expand_sparse(float* values, const int32_t* cols, int64_t batch, int64_t rows, int64_t n,
                       int32_t nnz, float scale, float* dense, int mode, void* stream);
+
+/*
+ * Two-transform Walsh-Hadamard expansion of sparse coefficients [QWHA §2.1:
+ * the form dW = H'^-1 F H^-1 of other Fourier-type adapters, here with
+ * Walsh-Hadamard transforms on both sides].
+ * values, cols: [batch, m, nnz] (fp32, int32); dense: fp32 [batch, m, n].
+ * mode 0: dense[b] = (H_m / sqrt m) scatter(values, cols)[b] H_n * scale
+ *   (duplicate columns add up);
+ * mode 1: values[b, r, k] = ((H_m / sqrt m) dense[b] H_n * scale)[r, cols[b, r, k]]
+ *   -- the gradient of mode 0 with respect to the values; dense is not
+ *   modified and the column transforms go to `workspace` (fp32, batch * m * n
+ *   elements, 16-byte aligned).
+ * m a power of two <= 2^24; n a power of two in [32, 32768]; 1 <= nnz <= n.
+ * Columns outside [0, n) are ignored (mode 0) / give 0 (mode 1).
+ */
+HIT_API int wht_expand_sparse_2d(float* values, const int32_t* cols, int64_t batch, int64_t m, int64_t n, int32_t nnz,
+                                 float scale, float* dense, int mode, void* workspace, size_t workspace_bytes,
+                                 void* stream);
+
+/*
+ * AdaAlloc around the sparse expansion [QWHA §2.2: a budget of coefficients
+ * is spread over the output channels (rows) in proportion to each channel's
+ * error with a minimum per channel; inside a channel the coefficients of
+ * largest magnitude are kept].
+ *
+ * row_norms: norms[r] = ||x[r, :n]||_2 (fp64 accumulation of the fp32
+ *   squares), x fp32 [rows, ldx] with n and ldx multiples of 4 and 16-byte
+ *   aligned rows; norms fp64 [rows] (device).  The channel error without
+ *   activations (the norm of a row of dW, equal to that of its coefficients).
+ *
+ * qwha_allocate (HOST pointers, no device work): counts[r] in [k_min, n] with
+ *   sum = budget (rows * k_min <= budget <= rows * n).  Every row gets k_min;
+ *   the remaining R units are split in proportion to err[r]: the share of an
+ *   uncapped row is (R' * err[r]) / S in float64, R' the units left for the
+ *   uncapped rows and S the left-to-right float64 sum of their errors; rows
+ *   whose share passes n - k_min are capped there and the rest re-split until
+ *   none passes; shares are rounded down and the leftover units go one each
+ *   to the largest fractional parts (ties to the lower row).  All-zero errors
+ *   split equally.  err must be finite and >= 0.
+ *
+ * qwha_select: per row r, the counts[r] = offsets[r+1] - offsets[r] entries of
+ *   largest |f[r, j]| (ties to the lower j), written in ascending j:
+ *   cols[offsets[r] + i] = j, values[...] = f[r, j].  f fp32 [rows, ldf]
+ *   (ldf >= n, multiple of 4, 16-byte aligned); offsets int64 [rows + 1],
+ *   cols int32 and values fp32 [offsets[rows]] (device).  n must be 1024,
+ *   2048, 4096 or 8192; counts must not exceed n.
+ */
+HIT_API int row_norms(const float* x, int64_t rows, int64_t n, int64_t ldx, double* norms, void* stream);
+HIT_API int qwha_allocate(const double* err, int64_t rows, int64_t budget, int64_t k_min, int64_t n, int64_t* counts);
+HIT_API int qwha_select(const float* f, int64_t rows, int64_t n, int64_t ldf, const int64_t* offsets, int32_t* cols,
+                        float* values, void* stream);
+
+/*
+ * HARP stage blocks from learnable parameters [HARP §2.2: each block is a
+ * learnable orthogonal factor times a fixed base mixer, B_c = Q(theta_c) G_b,
+ * Givens for b = 2, Cayley map (I - A)^-1 (I + A) for b > 2, all parameters
+ * zero = the fixed RHT; §2.4: int8 parameter storage].
+ * Builds every block of ONE stage of radix b (1 <= b <= 16) for `groups`
+ * groups, in the layout butterfly_apply reads: blocks [groups, b, b] fp32
+ * row-major (groups = L / b for the stage of a length-L transform).
+ *  - Parameters per block P = 0 (b = 1), 1 (b = 2: the angle phi of
+ *    Q = [[cos phi, -sin phi], [sin phi, cos phi]]), b (b - 1) / 2 (b > 2: A is
+ *    skew-symmetric with A[i][j] = theta_k, A[j][i] = -theta_k for i < j, pairs
+ *    k numbered row by row (0,1), (0,2), ..., (1,2), ...).
+ *  - Give exactly one of theta (fp32 [groups, P]) and theta_q (int8
+ *    [groups, P], standing for fp32(q) * theta_scale); both may be NULL for b = 1.
+ *  - mixer: fp32 [b, b] row-major orthogonal G_b; NULL means the normalized
+ *    Sylvester Hadamard H_b / sqrt(b), and is only allowed for powers of two.
+ *  - signs: NULL, or int8 [b * groups]: column k of block c is multiplied by
+ *    signs[k * groups + c], the sign of the input position that column reads
+ *    in the FIRST stage (t = 0) of a transform.  Folding the RHT's sign vector
+ *    into stage 0 this way makes butterfly_apply compute R(theta) diag(s) x,
+ *    and with transpose = 1 its inverse diag(s) R(theta)^T y.
+ * All pointers are device pointers.  Arithmetic in fp32 (Gauss-Jordan solve
+ * without pivoting: the symmetric part of I - A is the identity).
+ */
+HIT_API int harp_blocks(const float* theta, const int8_t* theta_q, float theta_scale, int64_t groups, int b,
+                        const float* mixer, const int8_t* signs, float* blocks, void* stream);
 
 /*
  * Fused RHT + group quantization without any allocation (no counterpart in

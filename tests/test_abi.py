@@ -171,3 +171,49 @@ def test_noalloc_checks_arguments_before_its_size_limit(lib):
     assert b"static scratch" in lib.hit_last_error()
     # no rows: nothing to do
     assert status(lib, na, FAKE, 0, 1024, 1024, 0, None, FAKE, 4, 128, FAKE, FAKE, None) == _lib.HIT_OK
+
+
+def test_harp_blocks_rejects_bad_arguments_on_host(lib):
+    h = "harp_blocks"
+    one = ctypes.c_float(1.0)
+    assert status(lib, h, FAKE, None, one, 4, 17, None, None, FAKE, None) == _lib.HIT_EUNSUPPORTED  # b > 16
+    assert status(lib, h, FAKE, None, one, 4, 0, None, None, FAKE, None) == _lib.HIT_EUNSUPPORTED
+    assert status(lib, h, FAKE, FAKE, one, 4, 4, None, None, FAKE, None) == _lib.HIT_EINVAL  # both thetas
+    assert status(lib, h, None, None, one, 4, 4, None, None, FAKE, None) == _lib.HIT_EINVAL  # neither
+    assert status(lib, h, FAKE, None, one, 4, 5, None, None, FAKE, None) == _lib.HIT_EINVAL  # radix 5 needs a mixer
+    assert status(lib, h, FAKE, None, one, 4, 4, None, None, None, None) == _lib.HIT_EINVAL  # no output
+    assert status(lib, h, FAKE, None, one, 4, 4, None, None, FAKE + 2, None) == _lib.HIT_EALIGN
+    assert status(lib, h, FAKE, None, one, 0, 4, None, None, FAKE, None) == _lib.HIT_OK  # no groups: nothing to do
+
+
+def test_mixed_rejects_bad_arguments_on_host(lib):
+    m = "rht_mixed_quantize_pack"
+    g = (ctypes.c_float * 25)(*([1.0] + [0.0] * 24))
+    gp = ctypes.cast(g, ctypes.c_void_p)
+    assert status(lib, m, FAKE, 4, 4096, 4096, None, gp, 4, 128, FAKE, FAKE, None) == _lib.HIT_EUNSUPPORTED
+    assert status(lib, m, FAKE, 4, 5120, 5120, None, gp, 3, 128, FAKE, FAKE, None) == _lib.HIT_EUNSUPPORTED
+    assert status(lib, m, FAKE, 4, 5120, 5120, None, gp, 4, 64, FAKE, FAKE, None) == _lib.HIT_EUNSUPPORTED
+    assert status(lib, m, FAKE, 4, 5120, 5120, None, None, 4, 128, FAKE, FAKE, None) == _lib.HIT_EINVAL
+    assert status(lib, m, FAKE, 4, 5120, 5121, None, gp, 4, 128, FAKE, FAKE, None) == _lib.HIT_EALIGN
+    assert status(lib, m, FAKE + 4, 4, 5120, 5120, None, gp, 4, 128, FAKE, FAKE, None) == _lib.HIT_EALIGN
+    assert status(lib, m, FAKE, 4, 5120, 5000, None, gp, 4, 128, FAKE, FAKE, None) == _lib.HIT_EINVAL
+    g[3] = float("nan")
+    assert status(lib, m, FAKE, 4, 5120, 5120, None, gp, 4, 128, FAKE, FAKE, None) == _lib.HIT_EINVAL
+    assert status(lib, m, FAKE, 0, 5120, 5120, None, gp, 4, 128, FAKE, FAKE, None) == _lib.HIT_OK
+
+
+def test_qwha_entry_points_reject_bad_arguments_on_host(lib):
+    assert status(lib, "qwha_select", FAKE, 4, 3000, 3000, FAKE, FAKE, FAKE, None) == _lib.HIT_EUNSUPPORTED
+    assert status(lib, "qwha_select", FAKE, 4, 4096, 4095, FAKE, FAKE, FAKE, None) == _lib.HIT_EINVAL
+    assert status(lib, "qwha_select", FAKE + 4, 4, 4096, 4096, FAKE, FAKE, FAKE, None) == _lib.HIT_EALIGN
+    assert status(lib, "qwha_select", FAKE, 0, 4096, 4096, FAKE, FAKE, FAKE, None) == _lib.HIT_OK
+    assert status(lib, "row_norms", FAKE, 4, 4098, 4098, FAKE, None) == _lib.HIT_EINVAL
+    assert status(lib, "row_norms", FAKE + 4, 4, 4096, 4096, FAKE, None) == _lib.HIT_EALIGN
+    w = "wht_expand_sparse_2d"
+    one = ctypes.c_float(1.0)
+    assert status(lib, w, FAKE, FAKE, 1, 300, 4096, 64, one, FAKE, 0, None, 0, None) == _lib.HIT_EUNSUPPORTED
+    assert status(lib, w, FAKE, FAKE, 1, 256, 4000, 64, one, FAKE, 0, None, 0, None) == _lib.HIT_EUNSUPPORTED
+    assert status(lib, w, FAKE, FAKE, 1, 256, 4096, 0, one, FAKE, 0, None, 0, None) == _lib.HIT_EINVAL
+    assert status(lib, w, FAKE, FAKE, 1, 256, 4096, 64, one, FAKE, 2, None, 0, None) == _lib.HIT_EINVAL
+    assert status(lib, w, FAKE, FAKE, 1, 256, 4096, 64, one, FAKE, 1, None, 0, None) == _lib.HIT_EWORKSPACE
+    assert status(lib, w, FAKE, FAKE, 0, 256, 4096, 64, one, FAKE, 0, None, 0, None) == _lib.HIT_OK

@@ -140,3 +140,18 @@ def test_two_sided_lowbit_workload_full_size(bits):
     mse_oracle = float(((rec - xb) ** 2).mean())
     mse_gpu = float(((host(y) - xb) ** 2).mean())
     assert abs(mse_gpu - mse_oracle) <= MSE_REL * mse_oracle, f"MSE {mse_gpu:.9e} vs oracle {mse_oracle:.9e}"
+
+
+@pytest.mark.parametrize("bits", [4, 2])
+def test_activation_per_token_quant_full_size(bits):
+    """Online activation path: bf16 8192 x 4096 tokens (0.5 * Student-t(3) with
+    1 % of the columns x20), RHT along the hidden dimension with Rademacher
+    signs, then one absmax scale per token (group = 4096), in the launch
+    configuration the benchmark times; every code against the oracle."""
+    d = synth.activation_rht()
+    xb = synth.bf16_bits_to_f32(d["x_bf16"])
+    codes, scales = hit.rht_quantize_pack(to_gpu_bf16(d["x_bf16"]), to_gpu_i8(d["signs"]), bits, 4096)
+    torch.cuda.synchronize()
+    assert scales.shape == (8192, 1)
+    ref = oq.quantize(oh.rht_rows(xb, d["signs"]), bits, 4096)
+    check_quant(codes, scales, ref, bits, 4096)
