@@ -7,6 +7,8 @@ ABI in include/hit.h; this package is a thin PyTorch binding over it.
 from ._lib import HitError, LIB_PATH, load  # noqa: F401
 from .api import (  # noqa: F401
     butterfly_apply,
+    butterfly_apply_tc,
+    butterfly_tc_workspace_bytes,
     codes_shape,
     dequant_inverse,
     harp_blocks,

@@ -29,6 +29,9 @@ SIGNATURES = {
     "rht_inverse": (_i32, [_vp, _vp, _i64, _i64, _i64, _i64, _i32, _i32, _vp, _i32, _vp, _sz, _vp]),
     "butterfly_apply": (_i32, [_vp, _vp, _i64, _i64, _i64, _i64, _i32, _i32, _i32, _vp, _vp, _vp, _i32, _i32,
                                _vp, _sz, _vp]),
+    "butterfly_apply_tc": (_i32, [_vp, _vp, _i64, _i64, _i64, _i64, _i32, _i32, _i32, _vp, _vp, _vp, _i32, _i32,
+                                  _vp, _sz, _vp]),
+    "butterfly_tc_workspace_bytes": (_sz, [_i64, _i64, _i32, _i32, _vp, _i32]),
     "rht_quantize_pack": (_i32, [_vp, _i64, _i64, _i64, _i32, _vp, _vp, _i32, _i32, _vp, _vp, _vp, _sz, _vp]),
     "rht_mixed_quantize_pack": (_i32, [_vp, _i64, _i64, _i64, _vp, _vp, _i32, _i32, _vp, _vp, _vp]),
     "dequant_inverse": (_i32, [_vp, _vp, _i64, _i64, _i32, _i32, _vp, _vp, _vp, _i64, _i32, _vp, _sz, _vp]),

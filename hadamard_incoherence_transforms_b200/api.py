@@ -364,3 +364,43 @@ def qwha_select(f, offsets, cols=None, values=None):
     call("qwha_select", f.data_ptr(), rows, n, f.stride(0), offsets.data_ptr(), cols.data_ptr(), values.data_ptr(),
          _stream(f.device))
     return cols, values
+
+
+def butterfly_tc_workspace_bytes(rows: int, n: int, radices, axis: int = 1, transpose: bool = False) -> int:
+    m = len(radices)
+    rad = (ctypes.c_int32 * m)(*[int(r) for r in radices])
+    return int(load().butterfly_tc_workspace_bytes(rows, n, axis, m, ctypes.cast(rad, ctypes.c_void_p),
+                                                   int(bool(transpose))))
+
+
+def butterfly_apply_tc(x, radices, blocks, axis: int = 1, transpose: bool = False, out=None, out_dtype=None,
+                       workspace=None):
+    """butterfly_apply on the tensor cores: bf16 input, window matrices composed on
+    the device, bf16 x bf16 -> fp32 products per pass, bf16 between passes."""
+    x = _mat(x, "x")
+    if x.dtype != torch.bfloat16:
+        raise ValueError("x must be bfloat16")
+    rows, n = x.shape
+    m = len(radices)
+    if len(blocks) != m:
+        raise ValueError("one block tensor per radix")
+    out_dtype = out_dtype or (out.dtype if out is not None else x.dtype)
+    if out is None:
+        out = torch.empty((rows, n), dtype=out_dtype, device=x.device)
+    _mat(out, "out")
+    for t, b in enumerate(blocks):
+        _cuda(b, f"blocks[{t}]")
+        if b.dtype != torch.float32 or b.dim() != 3 or not b.is_contiguous():
+            raise ValueError(f"blocks[{t}] must be contiguous float32 [G, b, b]")
+    rad = (ctypes.c_int32 * m)(*[int(r) for r in radices])
+    bptr = (ctypes.c_void_p * m)(*[b.data_ptr() for b in blocks])
+    ng = (ctypes.c_int64 * m)(*[int(b.shape[0]) for b in blocks])
+    need = butterfly_tc_workspace_bytes(rows, n, radices, axis, transpose)
+    ws = workspace
+    if ws is None and need > 0:
+        ws = torch.empty(need // 4 + 64, dtype=torch.float32, device=x.device)
+    call("butterfly_apply_tc", x.data_ptr(), out.data_ptr(), rows, n, x.stride(0), out.stride(0), _dt(x.dtype),
+         _dt(out_dtype), m, ctypes.cast(rad, ctypes.c_void_p), ctypes.cast(bptr, ctypes.c_void_p),
+         ctypes.cast(ng, ctypes.c_void_p), int(bool(transpose)), axis, _ptr(ws),
+         0 if ws is None else ws.numel() * ws.element_size(), _stream(x.device))
+    return out

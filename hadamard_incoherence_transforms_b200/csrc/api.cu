@@ -311,6 +311,7 @@ int hit_wait_timeouts(unsigned long long* count, int reset) {
   unsigned long long n = 0;
   e = hit::wait_timeouts_stream(&n, reset != 0);
   if (e == cudaSuccess) e = hit::wait_timeouts_mixed(&n, reset != 0);
+  if (e == cudaSuccess) e = hit::wait_timeouts_tc(&n, reset != 0);
   if (e != cudaSuccess) return cuda_status(e, "hit_wait_timeouts: counter read");
   if (count != nullptr) *count += n;
   if (n != 0)
@@ -446,6 +447,156 @@ int butterfly_apply(const void* x, void* y, int64_t rows, int64_t n, int64_t ldx
   return HIT_OK;
 }
 
+// ---------------------------------------------------------------------------
+// Tensor-core butterfly planning.  A pass is a run of consecutive stages (in
+// application order) whose digits form a range [dlo, dhi]; with P the product
+// of its radices and S_in the stride of digit dhi it mixes only the positions
+// of a window.  It runs on the tensor cores when its window matrix fits one
+// MMA tile:
+//   along rows (axis 1): S_in = 1 and P in {64, 128, 192, 256}: window = P
+//     contiguous positions;
+//   along columns (axis 0): P in {128, 256} (window = P positions at stride
+//     S_in), or S_in = 1 and P a divisor of 128 (window = 128 contiguous
+//     positions holding 128 / P groups: a block-diagonal matrix).
+// Any other run goes through the SIMT pass.
+// ---------------------------------------------------------------------------
+namespace {
+
+struct TcPlanPass {
+  bool tc = false;
+  int first = 0, count = 0;  // stages order[first .. first + count)
+  int Pw = 0;
+  int64_t step = 1;
+  hit::BflyPass simt;
+};
+
+bool tc_window(const int* order, int cnt, const int32_t* radices, const int64_t* S, int axis, int& Pw,
+               int64_t& step) {
+  int dlo = order[0], dhi = order[0];
+  for (int k = 1; k < cnt; ++k) {
+    dlo = order[k] < dlo ? order[k] : dlo;
+    dhi = order[k] > dhi ? order[k] : dhi;
+  }
+  if (dhi - dlo + 1 != cnt) return false;
+  int64_t P = 1;
+  for (int t = dlo; t <= dhi; ++t) P *= radices[t];
+  const int64_t s_in = S[dhi];
+  if (axis == 1) {
+    if (s_in != 1 || P % 64 != 0 || P > 256) return false;
+    Pw = int(P);
+    step = 1;
+    return true;
+  }
+  if (P == 128 || P == 256) {
+    Pw = int(P);
+    step = s_in;
+    return true;
+  }
+  if (s_in == 1 && P <= 128 && 128 % P == 0) {
+    Pw = 128;
+    step = 1;
+    return true;
+  }
+  return false;
+}
+
+// Passes of the tensor-core plan: from each stage, the longest run that is a
+// tensor-core window; otherwise a SIMT pass that stops before the next stage
+// at which a tensor-core run could start.
+bool plan_tc(int n_stages, const int32_t* radices, const int64_t* S, const float* const* blocks,
+             const int64_t* n_groups, int64_t len, int64_t outer, int axis, bool transpose, const int* order,
+             std::vector<TcPlanPass>& out) {
+  auto tc_from = [&](int i, int& cnt, int& Pw, int64_t& step) {
+    for (int j = n_stages; j > i; --j)
+      if (tc_window(order + i, j - i, radices, S, axis, Pw, step)) {
+        cnt = j - i;
+        return true;
+      }
+    return false;
+  };
+  int i = 0;
+  while (i < n_stages) {
+    TcPlanPass p;
+    int cnt = 0, Pw = 0;
+    int64_t step = 1;
+    if (tc_from(i, cnt, Pw, step)) {
+      p.tc = true;
+      p.first = i;
+      p.count = cnt;
+      p.Pw = Pw;
+      p.step = step;
+      // the window must tile the transform, and its matrix rows must fit one box
+      if (len % (int64_t(Pw) * step) != 0) return false;
+      out.push_back(p);
+      i += cnt;
+      continue;
+    }
+    int limit = n_stages;
+    for (int k = i + 1; k < n_stages; ++k) {
+      int c2 = 0, pw2 = 0;
+      int64_t st2 = 1;
+      if (tc_from(k, c2, pw2, st2)) {
+        limit = k;
+        break;
+      }
+    }
+    bool have = false;
+    for (int j = i; j < limit; ++j) {
+      hit::BflyPass cand;
+      if (!plan_pass(order + i, j - i + 1, radices, S, blocks, n_groups, len, outer, axis, transpose, cand)) break;
+      p.simt = cand;
+      have = true;
+    }
+    if (!have) return false;
+    p.tc = false;
+    p.first = i;
+    p.count = p.simt.ns;
+    out.push_back(p);
+    i += p.count;
+  }
+  return true;
+}
+
+size_t align256(size_t v) { return (v + 255) & ~size_t(255); }
+
+}  // namespace
+
+extern "C" {
+
+size_t butterfly_tc_workspace_bytes(int64_t rows, int64_t n, int axis, int n_stages, const int32_t* radices,
+                                    int transpose) {
+  if (rows <= 0 || n <= 0 || n_stages < 1 || n_stages > 16 || radices == nullptr) return 0;
+  const int64_t len = axis == 1 ? n : rows;
+  int64_t S[16], acc = 1;
+  for (int t = n_stages - 1; t >= 0; --t) {
+    if (radices[t] < 1) return 0;
+    S[t] = acc;
+    acc *= radices[t];
+  }
+  if (acc != len) return 0;
+  int order[16];
+  for (int i = 0; i < n_stages; ++i) order[i] = transpose ? n_stages - 1 - i : i;
+  size_t total = 0;
+  int passes = 0, i = 0;
+  while (i < n_stages) {
+    int Pw = 0;
+    int64_t step = 1;
+    int cnt = 0;
+    for (int j = n_stages; j > i; --j)
+      if (tc_window(order + i, j - i, radices, S, axis, Pw, step)) {
+        cnt = j - i;
+        break;
+      }
+    if (cnt > 0) total += align256(size_t(len) * size_t(Pw) * 2);
+    i += cnt > 0 ? cnt : 1;  // a bound: SIMT runs may merge several stages
+    ++passes;
+  }
+  const size_t inter = align256(size_t(rows) * size_t(n) * 2);
+  return total + (passes > 1 ? inter : 0) + (passes > 2 ? inter : 0);
+}
+
+}  // extern "C"
+
 static int check_quant_common(const char* fn, int64_t rows, int64_t n, int bits, int group) {
   if (rows < 0) return fail(HIT_EINVAL, "%s: rows < 0", fn);
   if (!is_pow2(n) || n < 32 || n > 32768) return fail(HIT_EUNSUPPORTED, "%s: n must be a power of two in [32, 32768]", fn);
@@ -505,6 +656,129 @@ int rht_quantize_pack(const void* x, int64_t rows, int64_t n, int64_t ldx, int d
   else if (bits == 3) e = hit::rows_quant_b3(logn, dt_rows, a, st);
   else e = hit::rows_quant_b2(logn, dt_rows, a, st);
   return cuda_status(e, fn);
+}
+
+int butterfly_apply_tc(const void* x, void* y, int64_t rows, int64_t n, int64_t ldx, int64_t ldy, int dtype_in,
+                       int dtype_out, int n_stages, const int32_t* radices, const float* const* blocks,
+                       const int64_t* n_groups, int transpose, int axis, void* workspace, size_t workspace_bytes,
+                       void* stream) {
+  const char* fn = "butterfly_apply_tc";
+  if (dtype_in != HIT_BF16) return fail(HIT_EUNSUPPORTED, "%s: the input must be bf16 (tensor-core operands)", fn);
+  if (!dtype_ok(dtype_out)) return fail(HIT_EUNSUPPORTED, "%s: unknown output dtype", fn);
+  if (rows < 0 || n < 1) return fail(HIT_EINVAL, "%s: bad shape", fn);
+  if (axis != 0 && axis != 1) return fail(HIT_EINVAL, "%s: axis must be 0 or 1", fn);
+  if (n_stages < 1 || n_stages > 16) return fail(HIT_EINVAL, "%s: n_stages must be 1..16", fn);
+  if (rows == 0) return ok();
+  if (radices == nullptr || blocks == nullptr || n_groups == nullptr)
+    return fail(HIT_EINVAL, "%s: radices, blocks and n_groups are required", fn);
+  if (x == nullptr || y == nullptr) return fail(HIT_EINVAL, "%s: x and y are required", fn);
+  if (x == y) return fail(HIT_EINVAL, "%s: x and y must not alias", fn);
+  if (ldx < n || ldy < n) return fail(HIT_EINVAL, "%s: leading dimension < n", fn);
+  if (!aligned(x, 16) || ldx % 8 != 0 || !aligned(y, 16) || (ldy * int64_t(esize(dtype_out))) % 16 != 0 || n % 8 != 0)
+    return fail(HIT_EALIGN, "%s: x, y and their row pitches must be 16-byte aligned and n a multiple of 8", fn);
+  if (rows > (int64_t(1) << 31) || n > (int64_t(1) << 31)) return fail(HIT_EUNSUPPORTED, "%s: too large", fn);
+  const int64_t len = axis == 1 ? n : rows;
+  int64_t prod = 1;
+  for (int t = 0; t < n_stages; ++t) {
+    if (radices[t] < 1 || radices[t] > 64) return fail(HIT_EUNSUPPORTED, "%s: radix %d outside 1..64", fn, radices[t]);
+    prod *= radices[t];
+    if (prod > (int64_t(1) << 40)) return fail(HIT_EINVAL, "%s: radices overflow", fn);
+  }
+  if (prod != len) return fail(HIT_EINVAL, "%s: radices multiply to %lld, transform length is %lld", fn,
+                               (long long)prod, (long long)len);
+  for (int t = 0; t < n_stages; ++t) {
+    if (blocks[t] == nullptr || !aligned(blocks[t], 4)) return fail(HIT_EINVAL, "%s: blocks[%d] missing or misaligned", fn, t);
+    if (n_groups[t] != 1 && n_groups[t] != len / radices[t])
+      return fail(HIT_EINVAL, "%s: n_groups[%d] must be 1 or %lld", fn, t, (long long)(len / radices[t]));
+  }
+  int64_t S[16];
+  {
+    int64_t acc = 1;
+    for (int t = n_stages - 1; t >= 0; --t) {
+      S[t] = acc;
+      acc *= radices[t];
+    }
+  }
+  int order[16];
+  for (int i = 0; i < n_stages; ++i) order[i] = transpose ? n_stages - 1 - i : i;
+  const int64_t outer = axis == 1 ? rows : n;
+  std::vector<TcPlanPass> plan;
+  if (!plan_tc(n_stages, radices, S, blocks, n_groups, len, outer, axis, transpose != 0, order, plan))
+    return fail(HIT_EUNSUPPORTED, "%s: no pass plan for this schedule", fn);
+  // workspace: window matrices of every tensor-core pass, then bf16 intermediates
+  const int np = static_cast<int>(plan.size());
+  std::vector<size_t> mat_ofs(np, 0);
+  size_t need = 0;
+  for (int q = 0; q < np; ++q)
+    if (plan[q].tc) {
+      mat_ofs[q] = need;
+      need += align256(size_t(len) * size_t(plan[q].Pw) * 2);
+    }
+  const size_t inter = align256(size_t(rows) * size_t(n) * 2);
+  const size_t inter_ofs = need;
+  need += (np > 1 ? inter : 0) + (np > 2 ? inter : 0);
+  if (need > 0 && (workspace == nullptr || workspace_bytes < need))
+    return fail(HIT_EWORKSPACE, "%s: needs %zu workspace bytes (butterfly_tc_workspace_bytes)", fn, need);
+  if (need > 0 && !aligned(workspace, 256)) return fail(HIT_EALIGN, "%s: workspace must be 256-byte aligned", fn);
+  uint8_t* ws = static_cast<uint8_t*>(workspace);
+  void* buf[2] = {ws + inter_ofs, ws + inter_ofs + inter};
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  for (int q = 0; q < np; ++q) {
+    const bool first = q == 0, last = q == np - 1;
+    const void* src = first ? x : buf[(q - 1) & 1];
+    const int64_t ld_src = first ? ldx : n;
+    void* dst = last ? y : buf[q & 1];
+    const int64_t ld_dst = last ? ldy : n;
+    const int dt_dst = last ? dtype_out : HIT_BF16;
+    TcPlanPass& p = plan[q];
+    if (!p.tc) {
+      p.simt.x = src;
+      p.simt.ldx = ld_src;
+      p.simt.y = dst;
+      p.simt.ldy = ld_dst;
+      const cudaError_t e = hit::launch_butterfly_pass(HIT_BF16, dt_dst, p.simt, st);
+      if (e != cudaSuccess) return cuda_status(e, fn);
+      continue;
+    }
+    hit::TcComposeArgs c;
+    c.Pw = p.Pw;
+    c.step = p.step;
+    c.ns = p.count;
+    for (int k = 0; k < p.count; ++k) {
+      const int t = order[p.first + k];
+      c.st[k].blocks = blocks[t];
+      c.st[k].b = radices[t];
+      c.st[k].stride = S[t];
+      c.st[k].shared_block = (n_groups[t] == 1 && len / radices[t] != 1) ? 1 : 0;
+      c.st[k].transpose = transpose ? 1 : 0;
+    }
+    auto* mats = reinterpret_cast<__nv_bfloat16*>(ws + mat_ofs[q]);
+    const int64_t n_windows = len / p.Pw;
+    cudaError_t e = hit::launch_bfly_compose(c, n_windows, mats, st);
+    if (e != cudaSuccess) return cuda_status(e, fn);
+    hit::TcPassArgs a;
+    a.cols = axis == 0 ? 1 : 0;
+    a.Pw = p.Pw;
+    a.K = p.Pw;
+    a.step = p.step;
+    a.L = len;
+    a.outer = rows;
+    a.ncols = n;
+    a.n_windows = static_cast<int>(n_windows);
+    if (axis == 1) {
+      a.N = p.Pw;
+      a.m_halves = 1;
+    } else {
+      a.N = 64;
+      a.m_halves = p.Pw / 128;
+    }
+    a.tmem_cols = a.N <= 32 ? 32 : (a.N <= 64 ? 64 : (a.N <= 128 ? 128 : 256));
+    a.y = dst;
+    a.ldy = ld_dst;
+    e = hit::launch_bfly_tc(a, src, ld_src, mats, dt_dst, st);
+    if (e != cudaSuccess) return cuda_status(e, fn);
+  }
+  return HIT_OK;
 }
 
 int rht_mixed_quantize_pack(const float* x, int64_t rows, int64_t n, int64_t ldx, const int8_t* signs,

@@ -1,6 +1,7 @@
 // Internal launcher interface between the C ABI (api.cu) and the kernel
 // translation units.  Host-side C++ only; no torch types anywhere.
 #pragma once
+#include <cuda_bf16.h>
 #include <cuda_runtime.h>
 #include <stddef.h>
 #include <stdint.h>
@@ -115,5 +116,38 @@ struct BflyPass {
   BflyStage st[kMaxPassStages];
 };
 cudaError_t launch_butterfly_pass(int dt_in, int dt_out, const BflyPass& p, cudaStream_t st);
+
+// Tensor-core butterfly passes (bfly_tc.cu).  A pass's window holds Pw
+// positions base(w) + p * step, base(w) = (w / step) * Pw * step + (w % step);
+// its stages are composed into one bf16 Pw x Pw matrix per window.
+struct TcStage {
+  const float* blocks = nullptr;  // [G, b, b] fp32 (or one shared block)
+  int b = 1;
+  int64_t stride = 1;             // digit stride S_t of the whole transform
+  int shared_block = 0;
+  int transpose = 0;              // use B^T
+};
+struct TcComposeArgs {
+  int Pw = 0;
+  int64_t step = 1;
+  int ns = 0;
+  TcStage st[kMaxPassStages];     // in application order
+};
+struct TcPassArgs {
+  int cols = 0;           // 0: row pass (windows along the contiguous dimension), 1: column pass
+  int Pw = 0, K = 0, N = 0;
+  int64_t step = 1;
+  int64_t L = 0;          // transform length
+  int64_t outer = 0;      // row pass: rows
+  int64_t ncols = 0;      // column pass: columns
+  int n_windows = 0, m_halves = 1, tmem_cols = 0;
+  int bytes_a = 0, bytes_b = 0;
+  void* y = nullptr;
+  int64_t ldy = 0;
+};
+cudaError_t launch_bfly_compose(const TcComposeArgs& a, int64_t n_windows, __nv_bfloat16* mats, cudaStream_t st);
+cudaError_t launch_bfly_tc(const TcPassArgs& a, const void* x, int64_t ldx, const __nv_bfloat16* mats, int dt_out,
+                           cudaStream_t st);
+cudaError_t wait_timeouts_tc(unsigned long long* count, bool reset);
 
 }  // namespace hit

@@ -121,8 +121,13 @@ __global__ void __launch_bounds__(StreamCfg<LOGN, Tin>::THREADS, 1) k_rows_strea
   uint32_t* sgn = reinterpret_cast<uint32_t*>(smem + 1024);
   uint8_t* slots = smem + 1024 + C::SIGNS;
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  SignLoad<G::N, C::NCW * 32> sl;
-  if (SIGNS && warp < C::NCW) sl.load(a.pre_signs, threadIdx.x);
+  // Launched as a programmatic dependent of the previous kernel in the stream:
+  // this CTA may start while that kernel's last CTAs still run (it only needs
+  // the SM), so it lets the next launch do the same, sets up its barriers,
+  // and waits for the previous kernel to complete (and its writes to become
+  // visible) before its first global-memory access.  Launched without that
+  // attribute, both instructions do nothing.
+  asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
   if (threadIdx.x == 0) {
     for (int s = 0; s < C::S; ++s) {
       for (int q = 0; q < C::NQ; ++q) mbar_init(&full[s * C::NQ + q], 1);
@@ -132,6 +137,9 @@ __global__ void __launch_bounds__(StreamCfg<LOGN, Tin>::THREADS, 1) k_rows_strea
     ticket[1] = 0;
     mbar_init_fence();
   }
+  asm volatile("griddepcontrol.wait;" ::: "memory");
+  SignLoad<G::N, C::NCW * 32> sl;
+  if (SIGNS && warp < C::NCW) sl.load(a.pre_signs, threadIdx.x);
   __syncthreads();
   const int64_t grid = gridDim.x;
   const int64_t nrows = a.rows > blockIdx.x ? (a.rows - blockIdx.x + grid - 1) / grid : 0;
@@ -286,8 +294,17 @@ cudaError_t launch_stream_k(const RowArgs& a, cudaStream_t st) {
   if ((e = cudaGetDevice(&dev)) != cudaSuccess) return e;
   if ((e = cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev)) != cudaSuccess) return e;
   const int64_t grid = a.rows < sms ? a.rows : sms;
-  kern<<<dim3(unsigned(grid)), C::THREADS, C::SMEM, st>>>(a);
-  return cudaGetLastError();
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(unsigned(grid));
+  cfg.blockDim = dim3(C::THREADS);
+  cfg.dynamicSmemBytes = C::SMEM;
+  cfg.stream = st;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  return cudaLaunchKernelEx(&cfg, kern, a);
 }
 
 // The sign flip is compiled in or out, so the row loop carries no branch on it.

@@ -157,6 +157,36 @@ HIT_API int butterfly_apply(const void* x, void* y, int64_t rows, int64_t n, int
                     void* workspace, size_t workspace_bytes, void* stream);
 
 /*
+ * The same rotation y = R x as butterfly_apply [HARP §2.1, §2.4: the stride
+ * stages as fused passes], on the tensor cores.  A run of consecutive stages
+ * whose digits vary inside a window of at most 256 positions is, restricted
+ * to each window, one dense matrix (the product of its blocks); the library
+ * composes these window matrices on the device (fp32, rounded once to bf16)
+ * and applies each pass as bf16 x bf16 products with fp32 accumulation
+ * (tcgen05 MMAs, operands staged by TMA).  Passes run on the tensor cores
+ * when the window is:
+ *   along rows (axis 1): the last digits with a product P in {64, 128, 192,
+ *     256} (P contiguous positions);
+ *   along columns (axis 0): digits with P in {128, 256} (positions at the
+ *     stride of the run's last digit), or the last digits with P dividing 128;
+ * other runs use the SIMT passes of butterfly_apply.  Data between passes is
+ * bf16, so results carry bf16 rounding per pass (use butterfly_apply for an
+ * fp32-accurate rotation).
+ * Arguments as butterfly_apply, with: dtype_in must be HIT_BF16; x and y must
+ * not alias; x, y 16-byte aligned, row pitches multiples of 16 bytes, n a
+ * multiple of 8; workspace (256-byte aligned) of at least
+ * butterfly_tc_workspace_bytes(rows, n, axis, n_stages, radices, transpose)
+ * bytes (the window matrices and the bf16 intermediates).
+ */
+HIT_API int butterfly_apply_tc(const void* x, void* y, int64_t rows, int64_t n, int64_t ldx, int64_t ldy,
+                               int dtype_in, int dtype_out, int n_stages, const int32_t* radices,
+                               const float* const* blocks, const int64_t* n_groups, int transpose, int axis,
+                               void* workspace, size_t workspace_bytes, void* stream);
+/* Workspace bound of butterfly_apply_tc (0 for invalid arguments); host arithmetic only. */
+HIT_API size_t butterfly_tc_workspace_bytes(int64_t rows, int64_t n, int axis, int n_stages, const int32_t* radices,
+                                            int transpose);
+
+/*
  * Fused RHT + group-wise symmetric absmax round-to-nearest quantization + code
  * packing [HARP §1, §5: incoherence processing before a blockwise quantizer].
  * x: [rows, n] (dtype_in, ldx).  One-sided (col_signs == NULL):

@@ -217,3 +217,33 @@ def test_qwha_entry_points_reject_bad_arguments_on_host(lib):
     assert status(lib, w, FAKE, FAKE, 1, 256, 4096, 64, one, FAKE, 2, None, 0, None) == _lib.HIT_EINVAL
     assert status(lib, w, FAKE, FAKE, 1, 256, 4096, 64, one, FAKE, 1, None, 0, None) == _lib.HIT_EWORKSPACE
     assert status(lib, w, FAKE, FAKE, 0, 256, 4096, 64, one, FAKE, 0, None, 0, None) == _lib.HIT_OK
+
+
+def test_butterfly_tc_host_checks_and_workspace(lib):
+    import ctypes as ct
+
+    def ws(rows, n, axis, radices, transpose=0):
+        r = (ct.c_int32 * len(radices))(*radices)
+        return lib.butterfly_tc_workspace_bytes(rows, n, axis, len(radices), ct.cast(r, ct.c_void_p), transpose)
+
+    # R_in of the butterfly workload: {2,3} on tensor cores (window 128), {0,1} SIMT, one bf16 intermediate
+    assert ws(4096, 14336, 1, (7, 16, 16, 8)) >= 14336 * 128 * 2 + 4096 * 14336 * 2
+    # R_out: {0,1} (window 256 at stride 16) and {2} (block-diagonal windows of 128)
+    assert ws(4096, 14336, 0, (16, 16, 16)) >= 4096 * 256 * 2 + 4096 * 128 * 2 + 4096 * 14336 * 2
+    assert ws(4096, 14336, 0, (16, 16, 15)) == 0  # radices do not multiply to the length
+    rad = (ct.c_int32 * 2)(16, 16)
+    blk = (ct.c_void_p * 2)(FAKE, FAKE)
+    ng = (ct.c_int64 * 2)(16, 16)
+    args = [ct.cast(rad, ct.c_void_p), ct.cast(blk, ct.c_void_p), ct.cast(ng, ct.c_void_p)]
+    t = "butterfly_apply_tc"
+    # fp32 input is refused (tensor-core operands are bf16)
+    assert status(lib, t, FAKE, FAKE + 0x100000, 8, 256, 256, 256, 0, 1, 2, *args, 0, 1, None, 0, None) == \
+        _lib.HIT_EUNSUPPORTED
+    # aliasing input and output
+    assert status(lib, t, FAKE, FAKE, 8, 256, 256, 256, 1, 1, 2, *args, 0, 1, None, 0, None) == _lib.HIT_EINVAL
+    # misaligned pitch
+    assert status(lib, t, FAKE, FAKE + 0x100000, 8, 256, 260, 256, 1, 1, 2, *args, 0, 1, None, 0, None) == \
+        _lib.HIT_EALIGN
+    # no workspace for the window matrices
+    assert status(lib, t, FAKE, FAKE + 0x100000, 8, 256, 256, 256, 1, 1, 2, *args, 0, 1, None, 0, None) == \
+        _lib.HIT_EWORKSPACE

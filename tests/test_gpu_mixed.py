@@ -40,7 +40,7 @@ def test_ragged_rows_no_signs_and_padded_pitch(rows):
     xg = to_gpu_f32(wide)[:, :5120]
     codes, scales = hit.rht_mixed_quantize_pack(xg, None, d["mixers"][5][0])
     torch.cuda.synchronize()
-    check_quant(codes, scales, oracle_codes(d, d["x"], None), 4, 5120)
+    check_quant(codes, scales, oracle_codes(d, d["x"], np.ones(5120, np.int8)), 4, 5120)
 
 
 def test_zero_rows_and_identity_mixer():
