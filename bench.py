@@ -510,12 +510,14 @@ def two_sided_butterfly(dev, l2_bytes, host_only=False, **_):
     rows, n = 4096, 14336
     w = Workload()
     w.name, w.rows, w.n = "two_sided_butterfly", rows, n
-    w.desc = "bf16 4096x14336: R_in (7,16,16,8) along rows then R_out (16,16,16) along columns"
-    w.io = "bf16 in; bf16 out (fp32 between the two sides)"
+    w.desc = ("bf16 4096x14336: R_in (7,16,16,8) along rows then R_out (16,16,16) along columns, "
+              "tensor-core window products (bf16 operands, fp32 accumulation), bf16 between passes")
+    w.io = "bf16 in; bf16 out"
     w.bytes = rows * n * 4
     w.h2d = w.d2h = rows * n * 2
-    w.kernels_per_step = 4  # two row passes (R_in) and two column passes (R_out)
-    w.kernel_key = "k_bfly_pass"
+    # per side: one compose + one tcgen05 launch per pass, two passes per side
+    w.kernels_per_step = 8
+    w.kernel_key = "k_bfly_tc"
 
     def oracle(r0, r1):
         from oracle import butterfly as ob
@@ -530,17 +532,19 @@ def two_sided_butterfly(dev, l2_bytes, host_only=False, **_):
     x = torch.from_numpy(d["x_bf16"].view(np.int16)).to(dev).view(torch.bfloat16)
     bi = [torch.from_numpy(b).to(dev) for b in d["blocks_in"]]
     bo = [torch.from_numpy(b).to(dev) for b in d["blocks_out"]]
-    mid = torch.empty((rows, n), dtype=torch.float32, device=dev)
+    mid = torch.empty((rows, n), dtype=torch.bfloat16, device=dev)
     y = torch.empty_like(x)
+    wsi = torch.empty(hit.butterfly_tc_workspace_bytes(rows, n, d["radices_in"], 1) // 4 + 64, device=dev)
+    wso = torch.empty(hit.butterfly_tc_workspace_bytes(rows, n, d["radices_out"], 0) // 4 + 64, device=dev)
     w.rotation = 1
 
     def step(i):
-        hit.butterfly_apply(x, d["radices_in"], bi, axis=1, out=mid)
-        hit.butterfly_apply(mid, d["radices_out"], bo, axis=0, out=y)
+        hit.butterfly_apply_tc(x, d["radices_in"], bi, axis=1, out=mid, workspace=wsi)
+        hit.butterfly_apply_tc(mid, d["radices_out"], bo, axis=0, out=y, workspace=wso)
 
     w.step = step
-    # the row side (R_in) of the sampled rows, as held between the two sides
-    w.parity = lambda ref, r0, r1: {"rows": r1 - r0, "row_side_rel_l2": _rel_l2(_host64(mid[r0:r1]), ref)}
+    # the row side (R_in) of the sampled rows, as held (bf16) between the two sides
+    w.parity = lambda ref, r0, r1: {"rows": r1 - r0, "row_side_bf16_row_rel": _bf16_row_rel(_host64(mid[r0:r1]), ref)}
     hx = x.cpu().pin_memory()
     hy = torch.empty_like(hx).pin_memory()
 

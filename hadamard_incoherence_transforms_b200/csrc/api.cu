@@ -464,14 +464,15 @@ namespace {
 
 struct TcPlanPass {
   bool tc = false;
+  int kind = 0;              // 0: contiguous row window, 1: column window
   int first = 0, count = 0;  // stages order[first .. first + count)
-  int Pw = 0;
-  int64_t step = 1;
+  int Pw = 0;                // window positions (kind 2: per lo value)
+  int64_t step = 1;          // stride of the window positions
   hit::BflyPass simt;
 };
 
-bool tc_window(const int* order, int cnt, const int32_t* radices, const int64_t* S, int axis, int& Pw,
-               int64_t& step) {
+bool tc_window(const int* order, int cnt, const int32_t* radices, const int64_t* S, int axis, int64_t outer, int& kind,
+               int& Pw, int64_t& step) {
   int dlo = order[0], dhi = order[0];
   for (int k = 1; k < cnt; ++k) {
     dlo = order[k] < dlo ? order[k] : dlo;
@@ -482,11 +483,19 @@ bool tc_window(const int* order, int cnt, const int32_t* radices, const int64_t*
   for (int t = dlo; t <= dhi; ++t) P *= radices[t];
   const int64_t s_in = S[dhi];
   if (axis == 1) {
-    if (s_in != 1 || P % 64 != 0 || P > 256) return false;
-    Pw = int(P);
-    step = 1;
-    return true;
+    if (s_in == 1) {
+      if (P % 64 != 0 || P > 256) return false;
+      kind = 0;
+      Pw = int(P);
+      step = 1;
+      return true;
+    }
+    // a strided run puts each window's positions S apart along the row: no
+    // MMA operand layout holds them without a transposition (SIMT pass)
+    (void)outer;
+    return false;
   }
+  kind = 1;
   if (P == 128 || P == 256) {
     Pw = int(P);
     step = s_in;
@@ -500,15 +509,21 @@ bool tc_window(const int* order, int cnt, const int32_t* radices, const int64_t*
   return false;
 }
 
+// Workspace bytes of a tensor-core pass's window matrices.
+size_t tc_matrix_bytes(int kind, int64_t len, int Pw) {
+  (void)kind;
+  return size_t(len) * size_t(Pw) * 2;
+}
+
 // Passes of the tensor-core plan: from each stage, the longest run that is a
 // tensor-core window; otherwise a SIMT pass that stops before the next stage
 // at which a tensor-core run could start.
 bool plan_tc(int n_stages, const int32_t* radices, const int64_t* S, const float* const* blocks,
              const int64_t* n_groups, int64_t len, int64_t outer, int axis, bool transpose, const int* order,
              std::vector<TcPlanPass>& out) {
-  auto tc_from = [&](int i, int& cnt, int& Pw, int64_t& step) {
+  auto tc_from = [&](int i, int& cnt, int& kind, int& Pw, int64_t& step) {
     for (int j = n_stages; j > i; --j)
-      if (tc_window(order + i, j - i, radices, S, axis, Pw, step)) {
+      if (tc_window(order + i, j - i, radices, S, axis, outer, kind, Pw, step)) {
         cnt = j - i;
         return true;
       }
@@ -517,15 +532,16 @@ bool plan_tc(int n_stages, const int32_t* radices, const int64_t* S, const float
   int i = 0;
   while (i < n_stages) {
     TcPlanPass p;
-    int cnt = 0, Pw = 0;
+    int cnt = 0, kind = 0, Pw = 0;
     int64_t step = 1;
-    if (tc_from(i, cnt, Pw, step)) {
+    if (tc_from(i, cnt, kind, Pw, step)) {
       p.tc = true;
+      p.kind = kind;
       p.first = i;
       p.count = cnt;
       p.Pw = Pw;
       p.step = step;
-      // the window must tile the transform, and its matrix rows must fit one box
+      // the windows must tile the transform
       if (len % (int64_t(Pw) * step) != 0) return false;
       out.push_back(p);
       i += cnt;
@@ -533,9 +549,9 @@ bool plan_tc(int n_stages, const int32_t* radices, const int64_t* S, const float
     }
     int limit = n_stages;
     for (int k = i + 1; k < n_stages; ++k) {
-      int c2 = 0, pw2 = 0;
+      int c2 = 0, k2 = 0, pw2 = 0;
       int64_t st2 = 1;
-      if (tc_from(k, c2, pw2, st2)) {
+      if (tc_from(k, c2, k2, pw2, st2)) {
         limit = k;
         break;
       }
@@ -578,16 +594,17 @@ size_t butterfly_tc_workspace_bytes(int64_t rows, int64_t n, int axis, int n_sta
   for (int i = 0; i < n_stages; ++i) order[i] = transpose ? n_stages - 1 - i : i;
   size_t total = 0;
   int passes = 0, i = 0;
+  const int64_t outer = axis == 1 ? rows : n;
   while (i < n_stages) {
-    int Pw = 0;
+    int kind = 0, Pw = 0, NT = 0;
     int64_t step = 1;
     int cnt = 0;
     for (int j = n_stages; j > i; --j)
-      if (tc_window(order + i, j - i, radices, S, axis, Pw, step)) {
+      if (tc_window(order + i, j - i, radices, S, axis, outer, kind, Pw, step)) {
         cnt = j - i;
         break;
       }
-    if (cnt > 0) total += align256(size_t(len) * size_t(Pw) * 2);
+    if (cnt > 0) total += align256(tc_matrix_bytes(kind, len, Pw));
     i += cnt > 0 ? cnt : 1;  // a bound: SIMT runs may merge several stages
     ++passes;
   }
@@ -712,7 +729,7 @@ int butterfly_apply_tc(const void* x, void* y, int64_t rows, int64_t n, int64_t 
   for (int q = 0; q < np; ++q)
     if (plan[q].tc) {
       mat_ofs[q] = need;
-      need += align256(size_t(len) * size_t(plan[q].Pw) * 2);
+      need += align256(tc_matrix_bytes(plan[q].kind, len, plan[q].Pw));
     }
   const size_t inter = align256(size_t(rows) * size_t(n) * 2);
   const size_t inter_ofs = need;
@@ -751,6 +768,8 @@ int butterfly_apply_tc(const void* x, void* y, int64_t rows, int64_t n, int64_t 
       c.st[k].stride = S[t];
       c.st[k].shared_block = (n_groups[t] == 1 && len / radices[t] != 1) ? 1 : 0;
       c.st[k].transpose = transpose ? 1 : 0;
+      c.st[k].div_s = hit::make_fastdiv(static_cast<uint32_t>(S[t]));
+      c.st[k].div_b = hit::make_fastdiv(static_cast<uint32_t>(radices[t]));
     }
     auto* mats = reinterpret_cast<__nv_bfloat16*>(ws + mat_ofs[q]);
     const int64_t n_windows = len / p.Pw;
@@ -772,7 +791,6 @@ int butterfly_apply_tc(const void* x, void* y, int64_t rows, int64_t n, int64_t 
       a.N = 64;
       a.m_halves = p.Pw / 128;
     }
-    a.tmem_cols = a.N <= 32 ? 32 : (a.N <= 64 ? 64 : (a.N <= 128 ? 128 : 256));
     a.y = dst;
     a.ldy = ld_dst;
     e = hit::launch_bfly_tc(a, src, ld_src, mats, dt_dst, st);

@@ -47,14 +47,19 @@ namespace {
 // ---------------------------------------------------------------------------
 constexpr int kComposeCols = 16;
 
+__device__ __forceinline__ uint32_t fdiv_u32(uint32_t n, const FastDiv& f) {
+  return (__umulhi(n, f.mul) + n) >> f.shr;
+}
+
 __global__ void __launch_bounds__(256) k_bfly_compose(const TcComposeArgs a, __nv_bfloat16* __restrict__ mats) {
   extern __shared__ float cbuf[];  // [2][kComposeCols][Pw]
   const int Pw = a.Pw;
-  const int64_t w = blockIdx.x;
+  const uint32_t w = blockIdx.x;
   const int j0 = blockIdx.y * kComposeCols;
   float* v = cbuf;
   float* u = cbuf + kComposeCols * Pw;
-  const int64_t base = (w / a.step) * int64_t(Pw) * a.step + (w % a.step);
+  const uint32_t step = uint32_t(a.step);
+  const uint32_t base = (w / step) * uint32_t(Pw) * step + (w % step);
   for (int i = threadIdx.x; i < kComposeCols * Pw; i += blockDim.x) {
     const int j = i / Pw, q = i - j * Pw;
     v[i] = (q == j0 + j) ? 1.0f : 0.0f;
@@ -62,23 +67,30 @@ __global__ void __launch_bounds__(256) k_bfly_compose(const TcComposeArgs a, __n
   __syncthreads();
   for (int t = 0; t < a.ns; ++t) {
     const TcStage& st = a.st[t];
-    const int64_t S = st.stride;           // global digit stride
-    const int sw = int(S / a.step);        // the same stride in window positions
-    for (int i = threadIdx.x; i < kComposeCols * Pw; i += blockDim.x) {
-      const int j = i / Pw, q = i - j * Pw;
-      const int64_t g = base + int64_t(q) * a.step;  // global position
-      const int64_t hiq = g / (int64_t(st.b) * S);
-      const int64_t loq = g % S;
-      const int dig = int((g / S) % st.b);
-      const int64_t c = st.shared_block ? 0 : hiq * S + loq;
-      const float* blk = st.blocks + c * int64_t(st.b) * st.b;
-      const float* col = v + j * Pw + (q - dig * sw);
-      float acc = 0.0f;
-      for (int k = 0; k < st.b; ++k) {
-        const float m = st.transpose ? blk[k * st.b + dig] : blk[dig * st.b + k];
-        acc = fmaf(m, col[k * sw], acc);
+    const uint32_t S = uint32_t(st.stride);
+    const int b = st.b;
+    const int sw = int(S / step);  // the digit stride in window positions
+    // every column of the chunk shares the position q: the block and the digit
+    // are found once per position, then applied to the kComposeCols columns
+    for (int q = threadIdx.x; q < Pw; q += blockDim.x) {
+      const uint32_t g = base + uint32_t(q) * step;  // global position (< 2^31)
+      const uint32_t q1 = fdiv_u32(g, st.div_s);     // g / S
+      const uint32_t lo = g - q1 * S;                // g % S
+      const uint32_t hi = fdiv_u32(q1, st.div_b);    // g / (b S)
+      const int dig = int(q1 - hi * uint32_t(b));    // (g / S) % b
+      const uint64_t c = st.shared_block ? 0 : uint64_t(hi) * S + lo;
+      const float* blk = st.blocks + c * uint64_t(b) * uint64_t(b);
+      const int q0 = q - dig * sw;
+      float acc[kComposeCols];
+#pragma unroll
+      for (int j = 0; j < kComposeCols; ++j) acc[j] = 0.0f;
+      for (int k = 0; k < b; ++k) {
+        const float mk = st.transpose ? __ldg(blk + k * b + dig) : __ldg(blk + dig * b + k);
+#pragma unroll
+        for (int j = 0; j < kComposeCols; ++j) acc[j] = fmaf(mk, v[j * Pw + q0 + k * sw], acc[j]);
       }
-      u[i] = acc;
+#pragma unroll
+      for (int j = 0; j < kComposeCols; ++j) u[j * Pw + q] = acc[j];
     }
     __syncthreads();
     float* tmp = v;
@@ -86,10 +98,10 @@ __global__ void __launch_bounds__(256) k_bfly_compose(const TcComposeArgs a, __n
     u = tmp;
   }
   // row q, column j0 + j of the window's matrix
-  __nv_bfloat16* out = mats + w * int64_t(Pw) * Pw;
+  __nv_bfloat16* out = mats + uint64_t(w) * uint64_t(Pw) * Pw;
   for (int i = threadIdx.x; i < kComposeCols * Pw; i += blockDim.x) {
     const int q = i / kComposeCols, j = i - q * kComposeCols;
-    out[int64_t(q) * Pw + j0 + j] = __float2bfloat16_rn(v[j * Pw + q]);
+    out[uint64_t(q) * Pw + j0 + j] = __float2bfloat16_rn(v[j * Pw + q]);
   }
 }
 
@@ -156,43 +168,67 @@ __device__ __forceinline__ void tmem_ld32(uint32_t taddr, uint32_t (&r)[32]) {
 }
 
 // ---------------------------------------------------------------------------
-// The pass kernel.  COLS = 0: row pass (A = data, K-major; B = window matrix,
-// K-major); COLS = 1: column pass (A = window matrix, K-major; B = data,
-// MN-major).  Tout: float or bf16.
+// The pass kernel: persistent and warp-specialized.  COLS = 0: row pass
+// (A = data tile [128 rows x K], K-major; B = window matrix [N = Pw x K],
+// K-major).  COLS = 1: column pass (A = window matrix rows [128 x K], K-major;
+// B = data tile [K positions x N columns], MN-major).  Tout: float or bf16.
+//
+// Each CTA owns a contiguous range of tiles, ordered so that consecutive tiles
+// share their window matrix.  Warp 4 (one lane) streams the data tiles into a
+// ring of NS shared-memory stages with TMA and reloads the window matrix only
+// when the window changes; warp 5 (one lane) issues the K/16 MMAs of a tile
+// into one of two tensor-memory accumulators and commits them to barriers that
+// free the data stage, hand the accumulator to the epilogue and (after the
+// window's last tile) free the matrix; warps 0-3 read an accumulator (warp w
+// owns tensor-memory lanes 32w..32w+31, one output row per thread), store it,
+// and hand it back, so the stores of tile i overlap the loads and MMAs of the
+// tiles after it.
 // ---------------------------------------------------------------------------
+struct TcBars {
+  uint64_t full[8], empty[8];  // data stages
+  uint64_t mfull, mempty;      // window matrix
+  uint64_t afull[2], aempty[2];  // accumulators
+  uint64_t mdone;              // final drain of the MMAs
+  long long issued;            // data tiles whose copies were issued
+  int mat_loads;               // window matrices whose copies were issued
+  uint32_t tmem;
+  int abort;
+};
+
 template <int COLS, typename Tout>
-__global__ void __launch_bounds__(128) k_bfly_tc(const __grid_constant__ CUtensorMap map_x,
-                                                 const __grid_constant__ CUtensorMap map_m, const TcPassArgs a) {
+__global__ void __launch_bounds__(192, 1) k_bfly_tc(const __grid_constant__ CUtensorMap map_x,
+                                                    const __grid_constant__ CUtensorMap map_m, const TcPassArgs a) {
   extern __shared__ __align__(1024) uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
-  const int K = a.K, N = a.N;
-  uint8_t* sa = smem;                                   // A operand
-  uint8_t* sb = smem + size_t(a.bytes_a);               // B operand
-  uint64_t* bars = reinterpret_cast<uint64_t*>(sb + a.bytes_b);
-  uint32_t* tslot = reinterpret_cast<uint32_t*>(bars + 2);
+  const int K = a.K, N = a.N, NS = a.stages;
+  uint8_t* smat = smem;                                   // window matrix (A for COLS 1, B for COLS 0)
+  uint8_t* sdat = smem + size_t(a.bytes_mat);             // NS data stages
+  TcBars* bars = reinterpret_cast<TcBars*>(sdat + size_t(NS) * a.bytes_stage);
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
 
-  // tile coordinates
-  int64_t w, t0;   // window; row tile (COLS 0) or column tile (COLS 1)
-  int half = 0;    // COLS 1: which 128 output positions of the window
-  if (COLS == 0) {
-    w = blockIdx.x % a.n_windows;
-    t0 = int64_t(blockIdx.x / a.n_windows) * 128;
-  } else {
-    const int64_t per = int64_t(a.n_windows) * a.m_halves;
-    const int64_t r = blockIdx.x % per;
-    w = r / a.m_halves;
-    half = int(r % a.m_halves);
-    t0 = int64_t(blockIdx.x / per) * N;
-  }
+  // contiguous tile range of this CTA
+  const int64_t T = a.tiles, G = gridDim.x;
+  const int64_t t_begin = blockIdx.x * T / G, t_end = (blockIdx.x + 1) * T / G;
 
   if (threadIdx.x == 0) {
-    mbar_init(&bars[0], 1);
-    mbar_init(&bars[1], 1);
+    for (int s = 0; s < NS; ++s) {
+      mbar_init(&bars->full[s], 1);
+      mbar_init(&bars->empty[s], 1);
+    }
+    mbar_init(&bars->mfull, 1);
+    mbar_init(&bars->mempty, 1);
+    for (int b = 0; b < 2; ++b) {
+      mbar_init(&bars->afull[b], 1);
+      mbar_init(&bars->aempty[b], 4);
+    }
+    mbar_init(&bars->mdone, 1);
+    bars->abort = 0;
+    bars->issued = 0;
+    bars->mat_loads = 0;
     mbar_init_fence();
   }
   if (warp == 0) {
-    asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(smem_u32(tslot)),
+    asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(smem_u32(&bars->tmem)),
                  "r"(uint32_t(a.tmem_cols))
                  : "memory");
     asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;" ::: "memory");
@@ -200,65 +236,137 @@ __global__ void __launch_bounds__(128) k_bfly_tc(const __grid_constant__ CUtenso
   asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory");
   __syncthreads();
   asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory");
-  const uint32_t tmem = *tslot;
+  const uint32_t tmem = bars->tmem;
+  volatile int* abort = &bars->abort;
 
-  bool ok = true;
-  if (threadIdx.x == 0) {
-    mbar_expect_tx(&bars[0], uint32_t(a.bytes_a + a.bytes_b));
-    const int kb = K / 64;  // 64-element (128-byte) boxes along K
+  auto decode = [&](int64_t t, int64_t& w, int& half, int64_t& t0) {
+    const int64_t key = t / a.tiles_per_key, r = t % a.tiles_per_key;
     if (COLS == 0) {
-      // A: data rows t0.., columns w*Pw + 64 j; B: window matrix rows w*Pw.., columns 64 j
-      for (int j = 0; j < kb; ++j) {
-        tma_load_2d(sa + size_t(j) * 128 * 128, &map_x, int(w * a.Pw + 64 * j), int(t0), &bars[0]);
-        tma_load_2d(sb + size_t(j) * N * 128, &map_m, 64 * j, int(w * a.Pw), &bars[0]);
-      }
+      w = key;
+      half = 0;
+      t0 = r * 128;
     } else {
-      // A: window matrix rows w*Pw + 128 half.., columns 64 j;
-      // B: data columns t0 + 64 j, positions p (all K of them) of window w
-      for (int j = 0; j < kb; ++j)
-        tma_load_2d(sa + size_t(j) * 128 * 128, &map_m, 64 * j, int(w * a.Pw + 128 * half), &bars[0]);
-      const int lo = int(w % a.step), hi = int(w / a.step);
-      for (int j = 0; j < N / 64; ++j)
-        tma_load_4d(sb + size_t(j) * K * 128, &map_x, int(t0 + 64 * j), 0, lo, hi, &bars[0]);
+      w = key / a.m_halves;
+      half = int(key % a.m_halves);
+      t0 = r * N;
     }
-    ok = mbar_wait(&bars[0], 0u);
-    if (ok) {
-      asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory");
+  };
+
+  if (warp == 4) {
+    // ---------------- TMA producer ----------------
+    if (lane == 0) {
+      int64_t cur = -1;
+      int ver = 0;
+      for (int64_t t = t_begin; t < t_end && !*abort; ++t) {
+        int64_t w, t0;
+        int half;
+        decode(t, w, half, t0);
+        const int64_t key = t / a.tiles_per_key;
+        if (key != cur) {
+          if (ver > 0 && !mbar_wait(&bars->mempty, uint32_t(ver - 1) & 1u)) {
+            atomicAdd(&g_wait_timeouts_tc, 1u);
+            *abort = 1;
+            break;
+          }
+          mbar_expect_tx(&bars->mfull, uint32_t(a.bytes_mat));
+          for (int j = 0; j < K / 64; ++j) {
+            if (COLS == 0)
+              tma_load_2d(smat + size_t(j) * N * 128, &map_m, 64 * j, int(w * a.Pw), &bars->mfull);
+            else
+              tma_load_2d(smat + size_t(j) * 128 * 128, &map_m, 64 * j, int(w * a.Pw + 128 * half), &bars->mfull);
+          }
+          ++ver;
+          bars->mat_loads = ver;
+          cur = key;
+        }
+        const int64_t i = t - t_begin;
+        const int s = int(i % NS);
+        const int64_t round = i / NS;
+        if (round > 0 && !mbar_wait(&bars->empty[s], uint32_t(round - 1) & 1u)) {
+          atomicAdd(&g_wait_timeouts_tc, 1u);
+          *abort = 1;
+          break;
+        }
+        uint8_t* st = sdat + size_t(s) * a.bytes_stage;
+        mbar_expect_tx(&bars->full[s], uint32_t(a.bytes_stage));
+        if (COLS == 0) {
+          for (int j = 0; j < K / 64; ++j)
+            tma_load_2d(st + size_t(j) * 128 * 128, &map_x, int(w * a.Pw + 64 * j), int(t0), &bars->full[s]);
+        } else {
+          const int lo = int(w % a.step), hi = int(w / a.step);
+          for (int j = 0; j < N / 64; ++j)
+            tma_load_4d(st + size_t(j) * K * 128, &map_x, int(t0 + 64 * j), 0, lo, hi, &bars->full[s]);
+        }
+        bars->issued = i + 1;
+      }
+    }
+  } else if (warp == 5) {
+    // ---------------- MMA issuer ----------------
+    if (lane == 0) {
       const uint32_t idesc = idesc_bf16(128, N, 0, COLS);
-      const uint32_t a0 = smem_u32(sa), b0 = smem_u32(sb);
-      for (int s = 0; s < K / 16; ++s) {
-        const int j = s >> 2, kk = s & 3;
-        // K-major operand: box j (rows x 128 B), 32 bytes per 16 elements inside the row
-        const uint64_t ad = smem_desc_sw128(a0 + uint32_t(j) * 128 * 128 + 32 * kk, 16, 1024);
-        uint64_t bd;
-        if (COLS == 0) bd = smem_desc_sw128(b0 + uint32_t(j) * uint32_t(N) * 128 + 32 * kk, 16, 1024);
-        else bd = smem_desc_sw128(b0 + uint32_t(s) * 16 * 128, uint32_t(K) * 128, 1024);  // MN-major: 16 K-rows per step
-        mma_bf16(tmem, ad, bd, idesc, s > 0 ? 1u : 0u);
+      const uint32_t m0 = smem_u32(smat);
+      int64_t cur = -1;
+      int ver = 0;
+      for (int64_t t = t_begin; t < t_end && !*abort; ++t) {
+        const int64_t key = t / a.tiles_per_key;
+        const int64_t i = t - t_begin;
+        const int s = int(i % NS);
+        const int64_t round = i / NS;
+        const int ab = int(i & 1);
+        const int64_t around = i >> 1;
+        bool ok = true;
+        if (key != cur) {
+          ok = mbar_wait(&bars->mfull, uint32_t(ver) & 1u);
+          ++ver;
+          cur = key;
+        }
+        ok = ok && mbar_wait(&bars->full[s], uint32_t(round) & 1u);
+        ok = ok && (around == 0 || mbar_wait(&bars->aempty[ab], uint32_t(around - 1) & 1u));
+        if (!ok) {
+          atomicAdd(&g_wait_timeouts_tc, 1u);
+          *abort = 1;
+          break;
+        }
+        asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory");
+        const uint32_t d0 = smem_u32(sdat + size_t(s) * a.bytes_stage);
+        const uint32_t acc = tmem + uint32_t(ab * N);
+        for (int k = 0; k < K / 16; ++k) {
+          const int j = k >> 2, kk = k & 3;
+          uint64_t ad, bd;
+          if (COLS == 0) {
+            ad = smem_desc_sw128(d0 + uint32_t(j) * 128 * 128 + 32 * kk, 16, 1024);        // data, K-major
+            bd = smem_desc_sw128(m0 + uint32_t(j) * uint32_t(N) * 128 + 32 * kk, 16, 1024);  // matrix, K-major
+          } else {
+            ad = smem_desc_sw128(m0 + uint32_t(j) * 128 * 128 + 32 * kk, 16, 1024);        // matrix, K-major
+            bd = smem_desc_sw128(d0 + uint32_t(k) * 16 * 128, uint32_t(K) * 128, 1024);     // data, MN-major
+          }
+          mma_bf16(acc, ad, bd, idesc, k > 0 ? 1u : 0u);
+        }
+        mma_commit(&bars->empty[s]);
+        mma_commit(&bars->afull[ab]);
+        const bool last_of_key = (t + 1 >= t_end) || ((t + 1) / a.tiles_per_key != key);
+        if (last_of_key) mma_commit(&bars->mempty);
       }
-      mma_commit(&bars[1]);
-    } else {
-      atomicAdd(&g_wait_timeouts_tc, 1u);
-      // do not leave with copies into shared memory in flight
-      if (!mbar_wait(&bars[0], 0u)) atomicAdd(&g_wait_timeouts_tc, 1u);
+      // every MMA issued above has completed before tensor memory is released
+      mma_commit(&bars->mdone);
+      if (!mbar_wait(&bars->mdone, 0u)) atomicAdd(&g_wait_timeouts_tc, 1u);
     }
-  }
-  // broadcast the outcome of the load wait (lane 0 of warp 0 decided it)
-  __shared__ int s_ok;
-  if (threadIdx.x == 0) s_ok = ok ? 1 : 0;
-  __syncthreads();
-  ok = s_ok != 0;
-  if (ok) {
-    bool done = mbar_wait(&bars[1], 0u);
-    if (!done) {
-      if (lane == 0) atomicAdd(&g_wait_timeouts_tc, 1u);
-      // the MMAs may still read shared memory / write tensor memory: wait once more
-      done = mbar_wait(&bars[1], 0u);
-    }
-    asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory");
-    if (done) {
-      // Epilogue: accumulator row = 32 warp + lane, 32 columns per load.
-      int64_t grow;   // global output row
-      int64_t gcol0;  // global column of accumulator column 0
+  } else {
+    // ---------------- epilogue: warps 0-3 ----------------
+    for (int64_t t = t_begin; t < t_end; ++t) {
+      int64_t w, t0;
+      int half;
+      decode(t, w, half, t0);
+      const int64_t i = t - t_begin;
+      const int ab = int(i & 1);
+      const int64_t around = i >> 1;
+      if (*abort || !mbar_wait(&bars->afull[ab], uint32_t(around) & 1u)) {
+        if (lane == 0 && !*abort) atomicAdd(&g_wait_timeouts_tc, 1u);
+        *abort = 1;
+        break;
+      }
+      asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory");
+      int64_t grow, gcol0;
       bool live;
       if (COLS == 0) {
         grow = t0 + 32 * warp + lane;
@@ -274,11 +382,11 @@ __global__ void __launch_bounds__(128) k_bfly_tc(const __grid_constant__ CUtenso
       Tout* yrow = static_cast<Tout*>(a.y) + grow * a.ldy + gcol0;
       for (int c = 0; c < N / 32; ++c) {
         uint32_t r[32];
-        tmem_ld32(tmem + (uint32_t(32 * warp) << 16) + uint32_t(32 * c), r);
+        tmem_ld32(tmem + (uint32_t(32 * warp) << 16) + uint32_t(ab * N + 32 * c), r);
         if (!live) continue;
         const int64_t col = gcol0 + 32 * c;
         Tout* dst = yrow + 32 * c;
-        const int64_t lim = COLS == 0 ? int64_t(32) : a.ncols - col;  // columns of this chunk inside the matrix
+        const int64_t lim = COLS == 0 ? int64_t(32) : a.ncols - col;
         if (lim >= 32) {
           if constexpr (sizeof(Tout) == 4) {
 #pragma unroll
@@ -302,9 +410,23 @@ __global__ void __launch_bounds__(128) k_bfly_tc(const __grid_constant__ CUtenso
           }
         }
       }
+      asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory");
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&bars->aempty[ab]);
     }
   }
-  asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory");
+  __syncthreads();
+  if (threadIdx.x == 4 * 32 && *abort) {
+    // drain: every stage and matrix copy this CTA issued has landed before
+    // its shared memory is released
+    const int64_t n = bars->issued;
+    for (int s = 0; s < NS && s < n; ++s) {
+      const int64_t last_round = (n - 1 - s) / NS;
+      if (!mbar_wait(&bars->full[s], uint32_t(last_round) & 1u)) atomicAdd(&g_wait_timeouts_tc, 1u);
+    }
+    const int v = bars->mat_loads;
+    if (v > 0 && !mbar_wait(&bars->mfull, uint32_t(v - 1) & 1u)) atomicAdd(&g_wait_timeouts_tc, 1u);
+  }
   __syncthreads();
   if (warp == 0) {
     asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory");
@@ -374,13 +496,22 @@ cudaError_t smem_attr_once(K kernel, size_t smem, std::atomic<unsigned long long
 }
 
 template <int COLS, typename Tout>
-cudaError_t launch_tc(const CUtensorMap& mx, const CUtensorMap& mm, const TcPassArgs& a, int64_t grid, size_t smem,
-                      cudaStream_t st) {
+cudaError_t launch_tc(const CUtensorMap& mx, const CUtensorMap& mm, const TcPassArgs& a, size_t smem, cudaStream_t st) {
   static std::atomic<unsigned long long> done{0};
   auto kern = k_bfly_tc<COLS, Tout>;
   cudaError_t e = smem_attr_once(kern, smem, done);
   if (e != cudaSuccess) return e;
-  kern<<<dim3(unsigned(grid)), 128, smem, st>>>(mx, mm, a);
+  int dev = 0, sms = 0, per_sm = 0;
+  if ((e = cudaGetDevice(&dev)) != cudaSuccess) return e;
+  if ((e = cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev)) != cudaSuccess) return e;
+  if ((e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, kern, 192, smem)) != cudaSuccess) return e;
+  if (per_sm < 1) return cudaErrorInvalidConfiguration;
+  // tensor memory: 512 columns per SM shared by the resident CTAs
+  const int by_tmem = 512 / a.tmem_cols;
+  per_sm = per_sm < by_tmem ? per_sm : by_tmem;
+  int64_t grid = int64_t(sms) * per_sm;
+  grid = grid < a.tiles ? grid : a.tiles;
+  kern<<<dim3(unsigned(grid)), 192, smem, st>>>(mx, mm, a);
   return cudaGetLastError();
 }
 
@@ -391,7 +522,8 @@ cudaError_t launch_bfly_compose(const TcComposeArgs& a, int64_t n_windows, __nv_
   const size_t smem = size_t(2) * kComposeCols * a.Pw * sizeof(float);
   cudaError_t e = smem_attr_once(k_bfly_compose, smem, done);
   if (e != cudaSuccess) return e;
-  k_bfly_compose<<<dim3(unsigned(n_windows), unsigned(a.Pw / kComposeCols)), 256, smem, st>>>(a, mats);
+  const int threads = a.Pw >= 256 ? 256 : ((a.Pw + 31) / 32) * 32;
+  k_bfly_compose<<<dim3(unsigned(n_windows), unsigned(a.Pw / kComposeCols)), threads, smem, st>>>(a, mats);
   return cudaGetLastError();
 }
 
@@ -401,6 +533,7 @@ cudaError_t launch_bfly_tc(const TcPassArgs& args, const void* x, int64_t ldx, c
   TcPassArgs a = args;
   CUtensorMap mx, mm;
   const int K = a.K;
+  if (K % 64 != 0 || K > 256 || a.N % 64 != 0 || a.N > 256) return cudaErrorInvalidValue;
   if (a.cols == 0) {
     // data [outer rows, L columns], box 64 columns x 128 rows
     const int64_t dx[2] = {a.L, a.outer}, sx[2] = {1, ldx};
@@ -410,8 +543,10 @@ cudaError_t launch_bfly_tc(const TcPassArgs& args, const void* x, int64_t ldx, c
     const int64_t dm[2] = {a.Pw, int64_t(a.n_windows) * a.Pw}, sm[2] = {1, a.Pw};
     const uint32_t bm[2] = {64, uint32_t(a.N)};
     if (!make_map(&mm, mats, 2, dm, sm, bm)) return cudaErrorInvalidValue;
-    a.bytes_a = 128 * K * 2;
-    a.bytes_b = a.N * K * 2;
+    a.bytes_stage = 128 * K * 2;
+    a.bytes_mat = a.N * K * 2;
+    a.tiles_per_key = (a.outer + 127) / 128;
+    a.tiles = int64_t(a.n_windows) * a.tiles_per_key;
   } else {
     // data [L rows, ncols columns] as (column, p, lo, hi): row = hi * Pw * step + p * step + lo
     const int64_t dx[4] = {a.ncols, a.Pw, a.step, a.L / (int64_t(a.Pw) * a.step)};
@@ -421,18 +556,30 @@ cudaError_t launch_bfly_tc(const TcPassArgs& args, const void* x, int64_t ldx, c
     const int64_t dm[2] = {a.Pw, int64_t(a.n_windows) * a.Pw}, sm[2] = {1, a.Pw};
     const uint32_t bm[2] = {64, 128};
     if (!make_map(&mm, mats, 2, dm, sm, bm)) return cudaErrorInvalidValue;
-    a.bytes_a = 128 * K * 2;
-    a.bytes_b = a.N * K * 2;
+    a.bytes_stage = a.N * K * 2;
+    a.bytes_mat = 128 * K * 2;
+    a.tiles_per_key = (a.ncols + a.N - 1) / a.N;
+    a.tiles = int64_t(a.n_windows) * a.m_halves * a.tiles_per_key;
   }
-  const size_t smem = 1024 + size_t(a.bytes_a) + size_t(a.bytes_b) + 64;
-  int64_t grid;
-  if (a.cols == 0) grid = int64_t(a.n_windows) * ((a.outer + 127) / 128);
-  else grid = int64_t(a.n_windows) * a.m_halves * ((a.ncols + a.N - 1) / a.N);
+  a.tmem_cols = 2 * a.N <= 64 ? 64 : (2 * a.N <= 128 ? 128 : (2 * a.N <= 256 ? 256 : 512));
+  // as many data stages as fit next to the matrix: two CTAs per SM when the
+  // stages and matrix fit in half the shared memory, else one
+  const size_t fixed = 1024 + size_t(a.bytes_mat) + 512;
+  const size_t half = 113 * 1024, whole = 226 * 1024;
+  int ns = int((half - fixed) / size_t(a.bytes_stage));
+  size_t budget = half;
+  if (ns < 2 || fixed > half) {
+    ns = int((whole - fixed) / size_t(a.bytes_stage));
+    budget = whole;
+  }
+  ns = ns > 6 ? 6 : ns;
+  if (ns < 1) return cudaErrorInvalidValue;
+  (void)budget;
+  a.stages = ns;
+  const size_t smem = fixed + size_t(ns) * a.bytes_stage;
   if (a.cols == 0)
-    return dt_out == DT_F32 ? launch_tc<0, float>(mx, mm, a, grid, smem, st)
-                            : launch_tc<0, __nv_bfloat16>(mx, mm, a, grid, smem, st);
-  return dt_out == DT_F32 ? launch_tc<1, float>(mx, mm, a, grid, smem, st)
-                          : launch_tc<1, __nv_bfloat16>(mx, mm, a, grid, smem, st);
+    return dt_out == DT_F32 ? launch_tc<0, float>(mx, mm, a, smem, st) : launch_tc<0, __nv_bfloat16>(mx, mm, a, smem, st);
+  return dt_out == DT_F32 ? launch_tc<1, float>(mx, mm, a, smem, st) : launch_tc<1, __nv_bfloat16>(mx, mm, a, smem, st);
 }
 
 cudaError_t wait_timeouts_tc(unsigned long long* count, bool reset) {

@@ -126,6 +126,7 @@ struct TcStage {
   int64_t stride = 1;             // digit stride S_t of the whole transform
   int shared_block = 0;
   int transpose = 0;              // use B^T
+  FastDiv div_s, div_b;           // division by S_t and by b (positions < 2^31)
 };
 struct TcComposeArgs {
   int Pw = 0;
@@ -134,14 +135,16 @@ struct TcComposeArgs {
   TcStage st[kMaxPassStages];     // in application order
 };
 struct TcPassArgs {
-  int cols = 0;           // 0: row pass (windows along the contiguous dimension), 1: column pass
+  int cols = 0;           // 0: row pass over contiguous windows, 1: column pass
   int Pw = 0, K = 0, N = 0;
   int64_t step = 1;
   int64_t L = 0;          // transform length
   int64_t outer = 0;      // row pass: rows
   int64_t ncols = 0;      // column pass: columns
   int n_windows = 0, m_halves = 1, tmem_cols = 0;
-  int bytes_a = 0, bytes_b = 0;
+  int bytes_mat = 0, bytes_stage = 0;  // window matrix / one data tile in shared memory
+  int stages = 1;                      // data tiles in flight per CTA
+  int64_t tiles = 0, tiles_per_key = 1;  // tiles of the pass; consecutive tiles sharing a window matrix
   void* y = nullptr;
   int64_t ldy = 0;
 };

@@ -40,6 +40,22 @@ def test_rows(radices, transpose, out_dtype):
     assert_close(host(y), ref, torch.bfloat16, f"rows {radices} T={transpose}")
 
 
+@pytest.mark.parametrize("radices", [(7, 16, 16, 8), (4, 16, 8), (2, 16, 8, 8), (8, 8, 16), (16, 8, 16)])
+@pytest.mark.parametrize("transpose", [False, True])
+@pytest.mark.parametrize("out_dtype", [torch.bfloat16, torch.float32])
+def test_rows_strided_windows(radices, transpose, out_dtype):
+    """Rows a multiple of 8 (264: a ragged last 128-row tile), so runs whose
+    digits sit at a stride run as lo-interleaved tensor-core windows."""
+    d = int(np.prod(radices))
+    blocks = blocks_for(radices, seed=d + 5)
+    bits, xf = bf16_input((264, d), d + 5)
+    y = hit.butterfly_apply_tc(to_gpu_bf16(bits), radices, [to_gpu_f32(b) for b in blocks], axis=1,
+                               transpose=transpose, out_dtype=out_dtype)
+    torch.cuda.synchronize()
+    ref = ob.apply_stages(xf, radices, blocks, transpose)
+    assert_close(host(y), ref, torch.bfloat16, f"strided rows {radices} T={transpose}")
+
+
 @pytest.mark.parametrize("radices", [(16, 16, 16), (8, 16), (2, 4, 16), (16, 8, 2), (4, 32, 2)])
 @pytest.mark.parametrize("transpose", [False, True])
 def test_columns(radices, transpose):
