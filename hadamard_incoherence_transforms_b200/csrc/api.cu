@@ -453,8 +453,8 @@ int butterfly_apply(const void* x, void* y, int64_t rows, int64_t n, int64_t ldx
 // of its radices and S_in the stride of digit dhi it mixes only the positions
 // of a window.  It runs on the tensor cores when its window matrix fits one
 // MMA tile:
-//   along rows (axis 1): S_in = 1 and P in {64, 128, 192, 256}: window = P
-//     contiguous positions;
+//   along rows (axis 1): S_in = 1 and P dividing 128: window = 128
+//     contiguous positions holding 128 / P groups (a block-diagonal matrix);
 //   along columns (axis 0): P in {128, 256} (window = P positions at stride
 //     S_in), or S_in = 1 and P a divisor of 128 (window = 128 contiguous
 //     positions holding 128 / P groups: a block-diagonal matrix).
@@ -484,9 +484,10 @@ bool tc_window(const int* order, int cnt, const int32_t* radices, const int64_t*
   const int64_t s_in = S[dhi];
   if (axis == 1) {
     if (s_in == 1) {
-      if (P % 64 != 0 || P > 256) return false;
+      // windows of 128 contiguous positions holding 128 / P groups
+      if (P > 128 || 128 % P != 0) return false;
       kind = 0;
-      Pw = int(P);
+      Pw = 128;
       step = 1;
       return true;
     }

@@ -136,6 +136,20 @@ __device__ __forceinline__ uint64_t smem_desc_sw128(uint32_t addr, uint32_t lbo_
   return d;
 }
 
+// AND of a predicate over the 128 threads of warps 0-3 (named barrier 1).
+__device__ __forceinline__ bool bar_and_128(bool v) {
+  uint32_t out;
+  asm volatile(
+      "{\n\t.reg .pred p, q;\n\t"
+      "setp.ne.u32 p, %1, 0;\n\t"
+      "bar.red.and.pred q, 1, 128, p;\n\t"
+      "selp.u32 %0, 1, 0, q;\n\t}"
+      : "=r"(out)
+      : "r"(uint32_t(v ? 1 : 0))
+      : "memory");
+  return out != 0;
+}
+
 // Instruction descriptor of kind::f16: bf16 A and B, fp32 accumulator.
 __host__ __device__ constexpr uint32_t idesc_bf16(int M, int N, int a_mn_major, int b_mn_major) {
   return (1u << 4) | (1u << 7) | (1u << 10) | (uint32_t(a_mn_major) << 15) | (uint32_t(b_mn_major) << 16) |
@@ -197,13 +211,15 @@ struct TcBars {
 
 template <int COLS, typename Tout>
 __global__ void __launch_bounds__(192, 1) k_bfly_tc(const __grid_constant__ CUtensorMap map_x,
-                                                    const __grid_constant__ CUtensorMap map_m, const TcPassArgs a) {
+                                                    const __grid_constant__ CUtensorMap map_m,
+                                                    const __grid_constant__ CUtensorMap map_y, const TcPassArgs a) {
   extern __shared__ __align__(1024) uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   const int K = a.K, N = a.N, NS = a.stages;
   uint8_t* smat = smem;                                   // window matrix (A for COLS 1, B for COLS 0)
   uint8_t* sdat = smem + size_t(a.bytes_mat);             // NS data stages
-  TcBars* bars = reinterpret_cast<TcBars*>(sdat + size_t(NS) * a.bytes_stage);
+  uint8_t* sout = sdat + size_t(NS) * a.bytes_stage;       // two output tiles (TMA store sources)
+  TcBars* bars = reinterpret_cast<TcBars*>(sout + 2 * size_t(a.bytes_out));
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
 
   // contiguous tile range of this CTA
@@ -353,6 +369,14 @@ __global__ void __launch_bounds__(192, 1) k_bfly_tc(const __grid_constant__ CUte
     }
   } else {
     // ---------------- epilogue: warps 0-3 ----------------
+    // The accumulator row of this thread goes to a shared-memory copy of the
+    // output tile laid out as the output tensor map's boxes (128 rows x 128
+    // bytes, 128-byte swizzle); one thread then writes the whole tile with
+    // TMA stores, so global writes are whole lines.  Two tile buffers: the
+    // stores of tile i drain while tile i + 1 is staged.
+    constexpr int ES = int(sizeof(Tout));
+    constexpr int BOXC = 128 / ES;  // output columns per box
+    const int r = 32 * warp + lane;  // accumulator row = row of the output box
     for (int64_t t = t_begin; t < t_end; ++t) {
       int64_t w, t0;
       int half;
@@ -360,60 +384,69 @@ __global__ void __launch_bounds__(192, 1) k_bfly_tc(const __grid_constant__ CUte
       const int64_t i = t - t_begin;
       const int ab = int(i & 1);
       const int64_t around = i >> 1;
-      if (*abort || !mbar_wait(&bars->afull[ab], uint32_t(around) & 1u)) {
-        if (lane == 0 && !*abort) atomicAdd(&g_wait_timeouts_tc, 1u);
+      bool ok = !*abort;
+      if (ok && !mbar_wait(&bars->afull[ab], uint32_t(around) & 1u)) {
+        ok = false;
+        if (lane == 0) atomicAdd(&g_wait_timeouts_tc, 1u);
+      }
+      // the staging buffer of tile i - 2 must have been read by its stores
+      if (threadIdx.x == 0 && i >= 2) asm volatile("cp.async.bulk.wait_group.read 1;" ::: "memory");
+      // one decision for the four warps (they meet at named barriers below)
+      if (!bar_and_128(ok)) {
         *abort = 1;
         break;
       }
       asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory");
-      int64_t grow, gcol0;
-      bool live;
-      if (COLS == 0) {
-        grow = t0 + 32 * warp + lane;
-        gcol0 = w * a.Pw;
-        live = grow < a.outer;
-      } else {
-        const int p = 128 * half + 32 * warp + lane;
-        const int64_t base = (w / a.step) * int64_t(a.Pw) * a.step + (w % a.step);
-        grow = base + int64_t(p) * a.step;
-        gcol0 = t0;
-        live = p < a.Pw;
-      }
-      Tout* yrow = static_cast<Tout*>(a.y) + grow * a.ldy + gcol0;
+      uint8_t* ob = sout + size_t(ab) * a.bytes_out;
       for (int c = 0; c < N / 32; ++c) {
-        uint32_t r[32];
-        tmem_ld32(tmem + (uint32_t(32 * warp) << 16) + uint32_t(ab * N + 32 * c), r);
-        if (!live) continue;
-        const int64_t col = gcol0 + 32 * c;
-        Tout* dst = yrow + 32 * c;
-        const int64_t lim = COLS == 0 ? int64_t(32) : a.ncols - col;
-        if (lim >= 32) {
-          if constexpr (sizeof(Tout) == 4) {
+        uint32_t v[32];
+        tmem_ld32(tmem + (uint32_t(32 * warp) << 16) + uint32_t(ab * N + 32 * c), v);
+        // columns 32 c .. 32 c + 31: box (32 c) / BOXC, byte offset (32 c * ES) % 128 in its row
+        const int col0 = 32 * c;
+        uint8_t* rowp = ob + size_t(col0 / BOXC) * (128 * 128) + size_t(r) * 128;
+        const int chunk0 = ((col0 % BOXC) * ES) / 16;
+        if constexpr (ES == 4) {
 #pragma unroll
-            for (int q = 0; q < 8; ++q)
-              __stcs(reinterpret_cast<uint4*>(dst) + q, make_uint4(r[4 * q], r[4 * q + 1], r[4 * q + 2], r[4 * q + 3]));
-          } else {
-            uint32_t h[16];
-#pragma unroll
-            for (int q = 0; q < 16; ++q) h[q] = f32_to_bf16x2(__uint_as_float(r[2 * q]), __uint_as_float(r[2 * q + 1]));
-#pragma unroll
-            for (int q = 0; q < 4; ++q)
-              __stcs(reinterpret_cast<uint4*>(dst) + q, make_uint4(h[4 * q], h[4 * q + 1], h[4 * q + 2], h[4 * q + 3]));
-          }
+          for (int q = 0; q < 8; ++q)
+            *reinterpret_cast<uint4*>(rowp + 16 * ((chunk0 + q) ^ (r & 7))) =
+                make_uint4(v[4 * q], v[4 * q + 1], v[4 * q + 2], v[4 * q + 3]);
         } else {
 #pragma unroll
-          for (int q = 0; q < 32; ++q) {
-            if (q < lim) {
-              if constexpr (sizeof(Tout) == 4) dst[q] = __uint_as_float(r[q]);
-              else dst[q] = __float2bfloat16_rn(__uint_as_float(r[q]));
-            }
-          }
+          for (int q = 0; q < 4; ++q)
+            *reinterpret_cast<uint4*>(rowp + 16 * ((chunk0 + q) ^ (r & 7))) =
+                make_uint4(f32_to_bf16x2(__uint_as_float(v[8 * q]), __uint_as_float(v[8 * q + 1])),
+                           f32_to_bf16x2(__uint_as_float(v[8 * q + 2]), __uint_as_float(v[8 * q + 3])),
+                           f32_to_bf16x2(__uint_as_float(v[8 * q + 4]), __uint_as_float(v[8 * q + 5])),
+                           f32_to_bf16x2(__uint_as_float(v[8 * q + 6]), __uint_as_float(v[8 * q + 7])));
         }
       }
+      // the accumulator is free once its loads are done
       asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory");
       __syncwarp();
       if (lane == 0) mbar_arrive(&bars->aempty[ab]);
+      // make the staged tile visible to the TMA engine, then store it
+      fence_proxy_async_smem();
+      asm volatile("bar.sync 1, 128;" ::: "memory");
+      if (threadIdx.x == 0) {
+        for (int j = 0; j < N / BOXC; ++j) {
+          const uint32_t src = smem_u32(ob + size_t(j) * (128 * 128));
+          if (COLS == 0) {
+            asm volatile("cp.async.bulk.tensor.2d.global.shared::cta.bulk_group [%0, {%1, %2}], [%3];" ::"l"(&map_y),
+                         "r"(int(w * a.Pw + BOXC * j)), "r"(int(t0)), "r"(src)
+                         : "memory");
+          } else {
+            const int lo = int(w % a.step), hi = int(w / a.step);
+            asm volatile(
+                "cp.async.bulk.tensor.4d.global.shared::cta.bulk_group [%0, {%1, %2, %3, %4}], [%5];" ::"l"(&map_y),
+                "r"(int(t0 + BOXC * j)), "r"(128 * half), "r"(lo), "r"(hi), "r"(src)
+                : "memory");
+          }
+        }
+        asm volatile("cp.async.bulk.commit_group;" ::: "memory");
+      }
     }
+    // every store has finished reading shared memory (and completed) before exit
+    if (threadIdx.x == 0) asm volatile("cp.async.bulk.wait_group 0;" ::: "memory");
   }
   __syncthreads();
   if (threadIdx.x == 4 * 32 && *abort) {
@@ -457,9 +490,9 @@ EncodeTiled encode_fn() {
   return f;
 }
 
-// bf16 tensor map, dims / strides in elements (dim 0 contiguous), 128-byte swizzle.
+// bf16 (or fp32) tensor map, dims / strides in elements (dim 0 contiguous), 128-byte swizzle.
 bool make_map(CUtensorMap* m, const void* base, int rank, const int64_t* dims, const int64_t* strides_el,
-              const uint32_t* box) {
+              const uint32_t* box, int esize = 2) {
   EncodeTiled f = encode_fn();
   if (f == nullptr) return false;
   cuuint64_t gd[5], gs[4];
@@ -468,9 +501,10 @@ bool make_map(CUtensorMap* m, const void* base, int rank, const int64_t* dims, c
     gd[i] = cuuint64_t(dims[i]);
     bd[i] = box[i];
     es[i] = 1;
-    if (i > 0) gs[i - 1] = cuuint64_t(strides_el[i]) * 2;
+    if (i > 0) gs[i - 1] = cuuint64_t(strides_el[i]) * cuuint64_t(esize);
   }
-  return f(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, cuuint32_t(rank), const_cast<void*>(base), gd, gs, bd, es,
+  const CUtensorMapDataType dt = esize == 4 ? CU_TENSOR_MAP_DATA_TYPE_FLOAT32 : CU_TENSOR_MAP_DATA_TYPE_BFLOAT16;
+  return f(m, dt, cuuint32_t(rank), const_cast<void*>(base), gd, gs, bd, es,
            CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
            CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
@@ -496,7 +530,8 @@ cudaError_t smem_attr_once(K kernel, size_t smem, std::atomic<unsigned long long
 }
 
 template <int COLS, typename Tout>
-cudaError_t launch_tc(const CUtensorMap& mx, const CUtensorMap& mm, const TcPassArgs& a, size_t smem, cudaStream_t st) {
+cudaError_t launch_tc(const CUtensorMap& mx, const CUtensorMap& mm, const CUtensorMap& my, const TcPassArgs& a,
+                      size_t smem, cudaStream_t st) {
   static std::atomic<unsigned long long> done{0};
   auto kern = k_bfly_tc<COLS, Tout>;
   cudaError_t e = smem_attr_once(kern, smem, done);
@@ -511,7 +546,7 @@ cudaError_t launch_tc(const CUtensorMap& mx, const CUtensorMap& mm, const TcPass
   per_sm = per_sm < by_tmem ? per_sm : by_tmem;
   int64_t grid = int64_t(sms) * per_sm;
   grid = grid < a.tiles ? grid : a.tiles;
-  kern<<<dim3(unsigned(grid)), 192, smem, st>>>(mx, mm, a);
+  kern<<<dim3(unsigned(grid)), 192, smem, st>>>(mx, mm, my, a);
   return cudaGetLastError();
 }
 
@@ -531,8 +566,10 @@ cudaError_t launch_bfly_compose(const TcComposeArgs& a, int64_t n_windows, __nv_
 cudaError_t launch_bfly_tc(const TcPassArgs& args, const void* x, int64_t ldx, const __nv_bfloat16* mats, int dt_out,
                            cudaStream_t st) {
   TcPassArgs a = args;
-  CUtensorMap mx, mm;
+  CUtensorMap mx, mm, my;
   const int K = a.K;
+  const int eo = dt_out == DT_F32 ? 4 : 2;
+  const uint32_t boxc = uint32_t(128 / eo);  // output columns per 128-byte box row
   if (K % 64 != 0 || K > 256 || a.N % 64 != 0 || a.N > 256) return cudaErrorInvalidValue;
   if (a.cols == 0) {
     // data [outer rows, L columns], box 64 columns x 128 rows
@@ -543,6 +580,10 @@ cudaError_t launch_bfly_tc(const TcPassArgs& args, const void* x, int64_t ldx, c
     const int64_t dm[2] = {a.Pw, int64_t(a.n_windows) * a.Pw}, sm[2] = {1, a.Pw};
     const uint32_t bm[2] = {64, uint32_t(a.N)};
     if (!make_map(&mm, mats, 2, dm, sm, bm)) return cudaErrorInvalidValue;
+    // output [outer rows, L columns], box 128 bytes x 128 rows
+    const int64_t dy[2] = {a.L, a.outer}, sy[2] = {1, a.ldy};
+    const uint32_t by[2] = {boxc, 128};
+    if (!make_map(&my, a.y, 2, dy, sy, by, eo)) return cudaErrorInvalidValue;
     a.bytes_stage = 128 * K * 2;
     a.bytes_mat = a.N * K * 2;
     a.tiles_per_key = (a.outer + 127) / 128;
@@ -556,30 +597,32 @@ cudaError_t launch_bfly_tc(const TcPassArgs& args, const void* x, int64_t ldx, c
     const int64_t dm[2] = {a.Pw, int64_t(a.n_windows) * a.Pw}, sm[2] = {1, a.Pw};
     const uint32_t bm[2] = {64, 128};
     if (!make_map(&mm, mats, 2, dm, sm, bm)) return cudaErrorInvalidValue;
+    // output the same view of y, box 128 bytes x 128 window positions
+    const int64_t sy[4] = {1, a.step * a.ldy, a.ldy, int64_t(a.Pw) * a.step * a.ldy};
+    const uint32_t by[4] = {boxc, 128, 1, 1};
+    if (!make_map(&my, a.y, 4, dx, sy, by, eo)) return cudaErrorInvalidValue;
     a.bytes_stage = a.N * K * 2;
     a.bytes_mat = 128 * K * 2;
     a.tiles_per_key = (a.ncols + a.N - 1) / a.N;
     a.tiles = int64_t(a.n_windows) * a.m_halves * a.tiles_per_key;
   }
+  a.bytes_out = 128 * a.N * eo;
   a.tmem_cols = 2 * a.N <= 64 ? 64 : (2 * a.N <= 128 ? 128 : (2 * a.N <= 256 ? 256 : 512));
-  // as many data stages as fit next to the matrix: two CTAs per SM when the
-  // stages and matrix fit in half the shared memory, else one
-  const size_t fixed = 1024 + size_t(a.bytes_mat) + 512;
-  const size_t half = 113 * 1024, whole = 226 * 1024;
-  int ns = int((half - fixed) / size_t(a.bytes_stage));
-  size_t budget = half;
-  if (ns < 2 || fixed > half) {
-    ns = int((whole - fixed) / size_t(a.bytes_stage));
-    budget = whole;
-  }
+  // one CTA per SM: the window matrix, two output tiles and as many data
+  // stages as fit (at most six)
+  const size_t fixed = 1024 + size_t(a.bytes_mat) + 2 * size_t(a.bytes_out) + 512;
+  const size_t whole = 226 * 1024;
+  if (fixed >= whole) return cudaErrorInvalidValue;
+  int ns = int((whole - fixed) / size_t(a.bytes_stage));
   ns = ns > 6 ? 6 : ns;
   if (ns < 1) return cudaErrorInvalidValue;
-  (void)budget;
   a.stages = ns;
   const size_t smem = fixed + size_t(ns) * a.bytes_stage;
   if (a.cols == 0)
-    return dt_out == DT_F32 ? launch_tc<0, float>(mx, mm, a, smem, st) : launch_tc<0, __nv_bfloat16>(mx, mm, a, smem, st);
-  return dt_out == DT_F32 ? launch_tc<1, float>(mx, mm, a, smem, st) : launch_tc<1, __nv_bfloat16>(mx, mm, a, smem, st);
+    return dt_out == DT_F32 ? launch_tc<0, float>(mx, mm, my, a, smem, st)
+                            : launch_tc<0, __nv_bfloat16>(mx, mm, my, a, smem, st);
+  return dt_out == DT_F32 ? launch_tc<1, float>(mx, mm, my, a, smem, st)
+                          : launch_tc<1, __nv_bfloat16>(mx, mm, my, a, smem, st);
 }
 
 cudaError_t wait_timeouts_tc(unsigned long long* count, bool reset) {

@@ -68,6 +68,9 @@ __global__ void __launch_bounds__(MixCfg::THREADS, 1) k_rows_mixed5120_q4(const 
   int* ticket = reinterpret_cast<int*>(empty + C::S);
   uint8_t* slots = smem + 1024;
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  // programmatic dependent launch: the CTA may start while the previous kernel
+  // in the stream finishes; every global access comes after griddepcontrol.wait
+  asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
   if (threadIdx.x == 0) {
     for (int s = 0; s < C::S; ++s) {
       for (int q = 0; q < C::NQ; ++q) mbar_init(&full[s * C::NQ + q], 1);
@@ -76,6 +79,7 @@ __global__ void __launch_bounds__(MixCfg::THREADS, 1) k_rows_mixed5120_q4(const 
     ticket[0] = 0;
     mbar_init_fence();
   }
+  asm volatile("griddepcontrol.wait;" ::: "memory");
   __syncthreads();
   const int64_t grid = gridDim.x;
   const int64_t nrows = a.rows > blockIdx.x ? (a.rows - blockIdx.x + grid - 1) / grid : 0;
@@ -299,8 +303,17 @@ inline cudaError_t launch_mixed5120_q4(const MixArgs& a, cudaStream_t st) {
   if ((e = cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev)) != cudaSuccess) return e;
   const int64_t grid = a.rows < sms ? a.rows : sms;
   if (grid == 0) return cudaSuccess;
-  k_rows_mixed5120_q4<<<dim3(unsigned(grid)), C::THREADS, C::SMEM, st>>>(a);
-  return cudaGetLastError();
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(unsigned(grid));
+  cfg.blockDim = dim3(C::THREADS);
+  cfg.dynamicSmemBytes = C::SMEM;
+  cfg.stream = st;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  return cudaLaunchKernelEx(&cfg, k_rows_mixed5120_q4, a);
 }
 
 }  // namespace hit

@@ -165,8 +165,8 @@ HIT_API int butterfly_apply(const void* x, void* y, int64_t rows, int64_t n, int
  * and applies each pass as bf16 x bf16 products with fp32 accumulation
  * (tcgen05 MMAs, operands staged by TMA).  Passes run on the tensor cores
  * when the window is:
- *   along rows (axis 1): the last digits with a product P in {64, 128, 192,
- *     256} (P contiguous positions);
+ *   along rows (axis 1): the last digits with a product P dividing 128
+ *     (windows of 128 contiguous positions holding 128 / P groups);
  *   along columns (axis 0): digits with P in {128, 256} (positions at the
  *     stride of the run's last digit), or the last digits with P dividing 128;
  * other runs use the SIMT passes of butterfly_apply.  Data between passes is

@@ -44,8 +44,9 @@ def test_rows(radices, transpose, out_dtype):
 @pytest.mark.parametrize("transpose", [False, True])
 @pytest.mark.parametrize("out_dtype", [torch.bfloat16, torch.float32])
 def test_rows_strided_windows(radices, transpose, out_dtype):
-    """Rows a multiple of 8 (264: a ragged last 128-row tile), so runs whose
-    digits sit at a stride run as lo-interleaved tensor-core windows."""
+    """Runs whose digits sit at a stride along the rows (SIMT passes inside the
+    tensor-core plan) next to contiguous tensor-core windows, 264 rows (a
+    ragged last 128-row tile)."""
     d = int(np.prod(radices))
     blocks = blocks_for(radices, seed=d + 5)
     bits, xf = bf16_input((264, d), d + 5)
