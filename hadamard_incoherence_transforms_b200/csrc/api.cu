@@ -312,6 +312,7 @@ int hit_wait_timeouts(unsigned long long* count, int reset) {
   e = hit::wait_timeouts_stream(&n, reset != 0);
   if (e == cudaSuccess) e = hit::wait_timeouts_mixed(&n, reset != 0);
   if (e == cudaSuccess) e = hit::wait_timeouts_tc(&n, reset != 0);
+  if (e == cudaSuccess) e = hit::wait_timeouts_strided(&n, reset != 0);
   if (e != cudaSuccess) return cuda_status(e, "hit_wait_timeouts: counter read");
   if (count != nullptr) *count += n;
   if (n != 0)
@@ -464,7 +465,7 @@ namespace {
 
 struct TcPlanPass {
   bool tc = false;
-  int kind = 0;              // 0: contiguous row window, 1: column window
+  int kind = 0;              // 0: contiguous row window, 1: column window, 2: strided two-digit row run
   int first = 0, count = 0;  // stages order[first .. first + count)
   int Pw = 0;                // window positions (kind 2: per lo value)
   int64_t step = 1;          // stride of the window positions
@@ -512,8 +513,7 @@ bool tc_window(const int* order, int cnt, const int32_t* radices, const int64_t*
 
 // Workspace bytes of a tensor-core pass's window matrices.
 size_t tc_matrix_bytes(int kind, int64_t len, int Pw) {
-  (void)kind;
-  return size_t(len) * size_t(Pw) * 2;
+  return kind == 2 ? 0 : size_t(len) * size_t(Pw) * 2;
 }
 
 // Passes of the tensor-core plan: from each stage, the longest run that is a
@@ -547,6 +547,23 @@ bool plan_tc(int n_stages, const int32_t* radices, const int64_t* S, const float
       out.push_back(p);
       i += cnt;
       continue;
+    }
+    // two adjacent digits along rows at a stride: the register-resident kernel
+    if (axis == 1 && i + 1 < n_stages) {
+      const int d0 = order[i], d1 = order[i + 1];
+      const int dh = d0 < d1 ? d0 : d1, dl = d0 < d1 ? d1 : d0;
+      const int64_t s_in = S[dl];
+      if (dl == dh + 1 && s_in % 8 == 0 && hit::strided_supported(radices[dh], radices[dl], 2, 4)) {
+        p.tc = true;
+        p.kind = 2;
+        p.first = i;
+        p.count = 2;
+        p.Pw = radices[dh] * radices[dl];
+        p.step = s_in;
+        out.push_back(p);
+        i += 2;
+        continue;
+      }
     }
     int limit = n_stages;
     for (int k = i + 1; k < n_stages; ++k) {
@@ -755,6 +772,27 @@ int butterfly_apply_tc(const void* x, void* y, int64_t rows, int64_t n, int64_t 
       p.simt.y = dst;
       p.simt.ldy = ld_dst;
       const cudaError_t e = hit::launch_butterfly_pass(HIT_BF16, dt_dst, p.simt, st);
+      if (e != cudaSuccess) return cuda_status(e, fn);
+      continue;
+    }
+    if (p.kind == 2) {
+      const int t0 = order[p.first], t1 = order[p.first + 1];
+      const int dh = t0 < t1 ? t0 : t1, dl = t0 < t1 ? t1 : t0;
+      hit::StridedArgs sa;
+      sa.x = src;
+      sa.y = dst;
+      sa.ldx = ld_src;
+      sa.ldy = ld_dst;
+      sa.rows = rows;
+      sa.s = p.step;
+      sa.n_hi = len / (int64_t(p.Pw) * p.step);
+      sa.blocks_h = blocks[dh];
+      sa.blocks_l = blocks[dl];
+      sa.shared_h = (n_groups[dh] == 1 && len / radices[dh] != 1) ? 1 : 0;
+      sa.shared_l = (n_groups[dl] == 1 && len / radices[dl] != 1) ? 1 : 0;
+      sa.transpose = transpose ? 1 : 0;
+      sa.h_first = t0 == dh ? 1 : 0;
+      const cudaError_t e = hit::launch_bfly_strided(radices[dh], radices[dl], HIT_BF16, dt_dst, sa, st);
       if (e != cudaSuccess) return cuda_status(e, fn);
       continue;
     }

@@ -1,0 +1,395 @@
+// Two-stage butterfly runs along rows whose digits sit at a stride (SIMT,
+// register resident, TMA tiles).
+//
+// HARP explainer, technical summary §2.1: each stage mixes, with a per-group
+// block, the coordinates that differ in one digit.  For a run of two adjacent
+// digits H (radix BH) and L (radix BL, even) whose positions in a row are
+//   g = hi * P * S + (iH * BL + iL) * S + lo,   P = BH * BL, S >= 8,
+// every (row, hi, lo) vector of P values is transformed on its own:
+//   stage on H: for each iL, x[. * BL + iL] <- B_H(c) x[. * BL + iL],
+//               c = (hi * BL + iL) * S + lo
+//   stage on L: for each iH, x[iH * BL + .] <- B_L(c) x[iH * BL + .],
+//               c = (hi * BH + iH) * S + lo
+// (the group numbering of the stage convention, digit removed).
+//
+// A CTA owns one (hi, 8-lo group) at a time and keeps the blocks of its eight
+// lo values in shared memory.  The data arrive as TMA boxes of 8 lo x (P + 1)
+// positions x R rows (dense 16-byte rows; the extra position skews the rows
+// across the shared-memory banks and is never used): one box loads while the
+// previous one is computed.  A lane holds half of the vector (the iL of one
+// parity, h, for every iH) of two rows of one lo: the stage on H is local, the
+// stage on L takes the partner half (lane ^ 16) by shuffles, and every
+// coefficient read from shared memory feeds both rows with packed fp32 FMAs.
+// Lane = h * 16 + rp * 8 + lo: the eight lo values of a half-warp read eight
+// different blocks laid out 4 words apart in the banks (one wavefront), and the
+// four (row, parity) pairs of a lo value read 16-byte rows in four distinct
+// bank groups.  Results go through a padded shared-memory tile to 16-byte
+// global stores.
+#include <cuda.h>
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+#include <atomic>
+#include <type_traits>
+
+#include "device.cuh"
+#include "internal.h"
+#include "rows_ops.cuh"
+
+namespace hit {
+
+__device__ unsigned int g_wait_timeouts_strided = 0;
+
+namespace {
+
+// Coefficients of one lo value in shared memory.  Stage on H: block iL at
+// iL BH BHP, entry (k, a) at k BHP + a = coefficient of output a from input k.
+// Stage on L: block iH at HF + iH BL BLP, entry (k, a) at k BLP + perm(a) with
+// the even outputs first, perm(a) = (a & 1) HL + a / 2, so that the outputs of
+// one parity are contiguous.  PER_LO is 4 mod 32 words: the blocks of eight lo
+// values start in eight different 4-bank groups.
+template <int BH, int BL>
+struct StridedBlocks {
+  static constexpr int BHP = (BH + 3) / 4 * 4;
+  static constexpr int BLP = (BL + 3) / 4 * 4;
+  static constexpr int HL = BL / 2;
+  static constexpr int HF = BL * BH * BHP + 4;
+  static constexpr int LF = BH * BL * BLP;
+  static constexpr int PER_LO = HF + LF;
+  static_assert(BL % 2 == 0, "the radix of L is split by parity");
+  static_assert(PER_LO % 32 == 4, "block layout must start the lo values in distinct bank groups");
+};
+
+// Stage the coefficients of one stage for the eight lo values of a group.  The
+// blocks of groups run0 + d * run_stride + l (l = 0..7) are eight consecutive
+// blocks in global memory for each of the NR run digits d, so every run is one
+// contiguous stretch of 8 B^2 floats: read coalesced, eight loads in flight per
+// thread.
+template <int B, int BP, int NR, bool PERM, int NT>
+__device__ __forceinline__ void stage_blocks(float* s_blk, int per_lo, int ofs, const float* blocks, int64_t run0,
+                                             int64_t run_stride, bool shared, bool transpose) {
+  constexpr int BB = B * B;
+  constexpr int RUN = 8 * BB;
+  constexpr int TOTAL = NR * RUN;
+  for (int base = 0; base < TOTAL; base += 8 * NT) {
+    float g[8];
+#pragma unroll
+    for (int u = 0; u < 8; ++u) {
+      const int i = base + int(threadIdx.x) + NT * u;
+      g[u] = 0.0f;
+      if (i < TOTAL) {
+        const int d = i / RUN, e = i - d * RUN;
+        g[u] = shared ? __ldg(blocks + e % BB) : __ldg(blocks + (run0 + int64_t(d) * run_stride) * BB + e);
+      }
+    }
+#pragma unroll
+    for (int u = 0; u < 8; ++u) {
+      const int i = base + int(threadIdx.x) + NT * u;
+      if (i < TOTAL) {
+        const int d = i / RUN, e = i - d * RUN;
+        const int l = e / BB, f = e - l * BB, rr = f / B, cc = f - rr * B;  // entry (rr, cc) of block l
+        const int k = transpose ? rr : cc, aa = transpose ? cc : rr;
+        const int col = PERM ? (aa & 1) * (B / 2) + (aa >> 1) : aa;
+        s_blk[l * per_lo + ofs + d * B * BP + k * BP + col] = g[u];
+      }
+    }
+  }
+}
+
+// Byte offset of element (row, p, lo) in a dense box (or tile) of 8 lo x
+// (P + 1) positions x rows with E-byte elements.
+template <int P, int E>
+__device__ __forceinline__ int box_offset(int row, int p, int lo) {
+  return ((row * (P + 1) + p) * 8 + lo) * E;
+}
+
+template <typename T>
+__device__ __forceinline__ float ld_elem(const uint8_t* p) {
+  if constexpr (std::is_same<T, float>::value) return *reinterpret_cast<const float*>(p);
+  else return __uint_as_float(uint32_t(*reinterpret_cast<const uint16_t*>(p)) << 16);
+}
+template <typename T>
+__device__ __forceinline__ void st_elem(uint8_t* p, float v) {
+  if constexpr (std::is_same<T, float>::value) *reinterpret_cast<float*>(p) = v;
+  else *reinterpret_cast<uint16_t*>(p) = __bfloat16_as_ushort(__float2bfloat16_rn(v));
+}
+
+// {o[q], o[q + 1]} += {c0, c1} * s for two rows sharing the coefficients
+__device__ __forceinline__ void fma2_rows(float c0, float c1, float s0, float s1, float& a0, float& a1, float& b0,
+                                          float& b1) {
+  fma_x2(c0, c1, s0, s0, a0, a1, a0, a1);
+  fma_x2(c0, c1, s1, s1, b0, b1, b0, b1);
+}
+
+// o_r[q] += b[q] * s_r (q < N, two rows) from 16- (or 8-) byte coefficient loads
+template <int N>
+__device__ __forceinline__ void axpy2(const float* b, float s0, float s1, float* o0, float* o1) {
+  if constexpr (N % 4 == 0 || N > 4) {
+#pragma unroll
+    for (int q4 = 0; q4 < (N + 3) / 4; ++q4) {
+      const float4 c = *reinterpret_cast<const float4*>(b + 4 * q4);
+      if (4 * q4 + 1 < N) {
+        fma2_rows(c.x, c.y, s0, s1, o0[4 * q4], o0[4 * q4 + 1], o1[4 * q4], o1[4 * q4 + 1]);
+      } else {
+        o0[4 * q4] = fmaf(c.x, s0, o0[4 * q4]);
+        o1[4 * q4] = fmaf(c.x, s1, o1[4 * q4]);
+      }
+      if (4 * q4 + 3 < N) {
+        fma2_rows(c.z, c.w, s0, s1, o0[4 * q4 + 2], o0[4 * q4 + 3], o1[4 * q4 + 2], o1[4 * q4 + 3]);
+      } else if (4 * q4 + 2 < N) {
+        o0[4 * q4 + 2] = fmaf(c.z, s0, o0[4 * q4 + 2]);
+        o1[4 * q4 + 2] = fmaf(c.z, s1, o1[4 * q4 + 2]);
+      }
+    }
+  } else {
+    static_assert(N == 2, "row segment of 2, 4k or more than 4 coefficients");
+    const float2 c = *reinterpret_cast<const float2*>(b);
+    fma2_rows(c.x, c.y, s0, s1, o0[0], o0[1], o1[0], o1[1]);
+  }
+}
+
+__device__ __forceinline__ void tma_load_3d(void* dst, const CUtensorMap* map, int c0, int c1, int c2, uint64_t* bar) {
+  asm volatile(
+      "cp.async.bulk.tensor.3d.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1, {%2, %3, %4}], [%5];" ::
+          "r"(smem_u32(dst)),
+      "l"(map), "r"(c0), "r"(c1), "r"(c2), "r"(smem_u32(bar))
+      : "memory");
+}
+template <int BH, int BL, int R, typename Tout>
+struct StridedGeom {
+  static constexpr int P = BH * BL;
+  static constexpr int NT = 8 * R;  // R / 2 row pairs x 8 lo x 2 halves
+  static constexpr int IN_BYTES = R * (P + 1) * 8 * 2;
+  static constexpr int OUT_BYTES = R * (P + 1) * 8 * int(sizeof(Tout));
+  static constexpr int IN_OFS = 0;  // 1024-byte aligned box
+  static constexpr int OUT_OFS = (IN_BYTES + 1023) / 1024 * 1024;
+  static constexpr int BLK_OFS = OUT_OFS + (OUT_BYTES + 15) / 16 * 16;
+  static constexpr int BAR_OFS = BLK_OFS + 8 * StridedBlocks<BH, BL>::PER_LO * 4;
+  static constexpr int SMEM = BAR_OFS + 16 + 1024;  // + slack to align the base
+};
+
+template <int BH, int BL, int R, typename Tout>
+__global__ void __launch_bounds__(8 * R, 1)
+    k_bfly_strided(const __grid_constant__ CUtensorMap map_x, const StridedArgs a) {
+  using SB = StridedBlocks<BH, BL>;
+  using G = StridedGeom<BH, BL, R, Tout>;
+  constexpr int P = G::P;
+  constexpr int HL = SB::HL;
+  constexpr int NV = BH * HL;  // values per lane and row
+  constexpr int EO = int(sizeof(Tout));
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* sm = smem_raw + ((1024u - (smem_u32(smem_raw) & 1023u)) & 1023u);
+  uint8_t* s_in = sm + G::IN_OFS;
+  uint8_t* s_out = sm + G::OUT_OFS;
+  float* s_blk = reinterpret_cast<float*>(sm + G::BLK_OFS);
+  uint64_t* full = reinterpret_cast<uint64_t*>(sm + G::BAR_OFS);
+
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int h = lane >> 4, rp = (lane >> 3) & 1, lo = lane & 7;
+  const int row0 = 4 * warp + 2 * rp;  // this lane's rows row0, row0 + 1 of the box
+  const int64_t S = a.s;
+  const int64_t groups8 = S / 8;
+  const int64_t n_keys = a.n_hi * groups8;
+  const int64_t row_tiles = (a.rows + R - 1) / R;
+  // CTA b works on keys ks, ks + kslots, ... and, for each, on row-tile range
+  // `part` of `parts`.  CTAs with consecutive b hold consecutive keys, so the
+  // ones in flight together read and write the same rows at the same time: the
+  // 16-byte rows of neighbouring lo groups fill the same DRAM lines while those
+  // are in L2.
+  const int64_t kslots = int64_t(gridDim.x) / a.parts;
+  const int64_t ks = blockIdx.x % kslots, part = blockIdx.x / kslots;
+  const int64_t rt_begin = part * row_tiles / a.parts, rt_end = (part + 1) * row_tiles / a.parts;
+  if (ks >= n_keys || rt_begin >= rt_end) return;
+  const __nv_bfloat16* x = static_cast<const __nv_bfloat16*>(a.x);
+  Tout* y = static_cast<Tout*>(a.y);
+  (void)x;
+  if (threadIdx.x == 0) {
+    mbar_init(full, 1);
+    mbar_init_fence();
+    mbar_expect_tx(full, uint32_t(G::IN_BYTES));
+    tma_load_3d(s_in, &map_x, int((ks % groups8) * 8), int((ks / groups8) * P), int(rt_begin * R), full);
+  }
+  uint32_t phase = 0;
+  const float* bl = s_blk + lo * SB::PER_LO;
+  for (int64_t key = ks; key < n_keys; key += kslots) {
+    const int64_t hi = key / groups8, lo0 = (key % groups8) * 8;
+    const int64_t col0 = hi * int64_t(P) * S + lo0;  // column of (iH, iL) = (0, 0), lo = lo0
+    __syncthreads();  // every lane done with the previous key's blocks
+    stage_blocks<BH, SB::BHP, BL, false, G::NT>(s_blk, SB::PER_LO, 0, a.blocks_h, hi * BL * S + lo0, S,
+                                                a.shared_h != 0, a.transpose != 0);
+    stage_blocks<BL, SB::BLP, BH, true, G::NT>(s_blk, SB::PER_LO, SB::HF, a.blocks_l, hi * BH * S + lo0, S,
+                                               a.shared_l != 0, a.transpose != 0);
+    __syncthreads();
+    for (int64_t rt = rt_begin; rt < rt_end; ++rt) {
+      const bool ok = mbar_wait(full, phase);
+      phase ^= 1u;
+      // this lane's half vectors: v_r[iH * HL + j] = position iH BL + 2 j + h of row row0 + r
+      float v0[NV], v1[NV];
+#pragma unroll
+      for (int iH = 0; iH < BH; ++iH)
+#pragma unroll
+        for (int j = 0; j < HL; ++j) {
+          const int p = iH * BL + 2 * j + h;
+          v0[iH * HL + j] = ld_elem<__nv_bfloat16>(s_in + box_offset<P, 2>(row0, p, lo));
+          v1[iH * HL + j] = ld_elem<__nv_bfloat16>(s_in + box_offset<P, 2>(row0 + 1, p, lo));
+        }
+      // every lane has read the box (and the previous tile's results have
+      // left the output tile): the next box may land
+      if (!__syncthreads_and(ok)) {
+        if (threadIdx.x == 0) atomicAdd(&g_wait_timeouts_strided, 1u);
+        return;
+      }
+      if (threadIdx.x == 0) {
+        int64_t nkey = key, nrt = rt + 1;
+        if (nrt == rt_end) {
+          nkey = key + kslots;
+          nrt = rt_begin;
+        }
+        if (nkey < n_keys) {
+          mbar_expect_tx(full, uint32_t(G::IN_BYTES));
+          tma_load_3d(s_in, &map_x, int((nkey % groups8) * 8), int((nkey / groups8) * P), int(nrt * R), full);
+        }
+      }
+      auto stage_h = [&]() {
+#pragma unroll
+        for (int j = 0; j < HL; ++j) {
+          const float* b = bl + (2 * j + h) * BH * SB::BHP;  // block iL = 2 j + h
+          float o0[BH], o1[BH];
+#pragma unroll
+          for (int q = 0; q < BH; ++q) o0[q] = o1[q] = 0.0f;
+#pragma unroll
+          for (int k = 0; k < BH; ++k) axpy2<BH>(b + k * SB::BHP, v0[k * HL + j], v1[k * HL + j], o0, o1);
+#pragma unroll
+          for (int q = 0; q < BH; ++q) {
+            v0[q * HL + j] = o0[q];
+            v1[q * HL + j] = o1[q];
+          }
+        }
+      };
+      auto stage_l = [&]() {
+#pragma unroll
+        for (int iH = 0; iH < BH; ++iH) {
+          float o0[HL], o1[HL];
+#pragma unroll
+          for (int q = 0; q < HL; ++q) o0[q] = o1[q] = 0.0f;
+          // outputs 2 q + h of block iH (contiguous after the column
+          // permutation); inputs 2 j + h (own) and 2 j + 1 - h (partner)
+          const float* b = bl + SB::HF + iH * BL * SB::BLP + h * HL;
+#pragma unroll
+          for (int j = 0; j < HL; ++j) {
+            const float own0 = v0[iH * HL + j], own1 = v1[iH * HL + j];
+            const float oth0 = __shfl_xor_sync(0xffffffffu, own0, 16);
+            const float oth1 = __shfl_xor_sync(0xffffffffu, own1, 16);
+            axpy2<HL>(b + (2 * j + h) * SB::BLP, own0, own1, o0, o1);
+            axpy2<HL>(b + (2 * j + 1 - h) * SB::BLP, oth0, oth1, o0, o1);
+          }
+#pragma unroll
+          for (int q = 0; q < HL; ++q) {
+            v0[iH * HL + q] = o0[q];
+            v1[iH * HL + q] = o1[q];
+          }
+        }
+      };
+      if (a.h_first) {
+        stage_h();
+        stage_l();
+      } else {
+        stage_l();
+        stage_h();
+      }
+#pragma unroll
+      for (int iH = 0; iH < BH; ++iH)
+#pragma unroll
+        for (int j = 0; j < HL; ++j) {
+          const int p = iH * BL + 2 * j + h;
+          st_elem<Tout>(s_out + box_offset<P, EO>(row0, p, lo), v0[iH * HL + j]);
+          st_elem<Tout>(s_out + box_offset<P, EO>(row0 + 1, p, lo), v1[iH * HL + j]);
+        }
+      __syncthreads();
+      // 16-byte global stores: piece (row, p) = the 8 lo values of one position
+      constexpr int WO = 8 * EO / 16;  // 16-byte words per piece
+      const int64_t r0 = rt * R;
+      for (int i = threadIdx.x; i < R * P * WO; i += G::NT) {
+        const int w = i % WO, pc = i / WO;
+        const int rr = pc / P, p = pc - rr * P;
+        const int64_t row = r0 + rr;
+        if (row >= a.rows) continue;
+        const uint4 val = *reinterpret_cast<const uint4*>(s_out + box_offset<P, EO>(rr, p, 0) + 16 * w);
+        __stcs(reinterpret_cast<uint4*>(y + row * a.ldy + col0 + int64_t(p) * S) + w, val);
+      }
+    }
+  }
+}
+
+template <int BH, int BL, int R, typename Tout>
+cudaError_t launch_strided_t(const StridedArgs& a, cudaStream_t st) {
+  using G = StridedGeom<BH, BL, R, Tout>;
+  static_assert(G::SMEM <= 227 * 1024, "shared memory");
+  static std::atomic<unsigned long long> done{0};
+  auto kern = k_bfly_strided<BH, BL, R, Tout>;
+  cudaError_t e = set_smem_attr(kern, G::SMEM, done);
+  if (e != cudaSuccess) return e;
+  int dev = 0, sms = 0;
+  if ((e = cudaGetDevice(&dev)) != cudaSuccess) return e;
+  if ((e = cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev)) != cudaSuccess) return e;
+  const int64_t n_keys = a.n_hi * (a.s / 8), row_tiles = (a.rows + R - 1) / R;
+  if (n_keys <= 0 || row_tiles <= 0) return cudaSuccess;
+  // input boxes: dim 0 = lo (S, contiguous), dim 1 = position P hi + p
+  // (stride S), dim 2 = row (stride ldx); a box of P + 1 positions reaches
+  // one position into the next hi block (or past the end: zero fill)
+  const int64_t len = a.n_hi * int64_t(G::P) * a.s;
+  CUtensorMap mx;
+  const int64_t dims[3] = {a.s, len / a.s, a.rows};
+  const int64_t sx[3] = {1, a.s, a.ldx};
+  const uint32_t box[3] = {8u, uint32_t(G::P + 1), uint32_t(R)};
+  if (!make_tensor_map(&mx, a.x, 3, dims, sx, box, 2, false)) return cudaErrorInvalidValue;
+  StridedArgs b = a;
+  int64_t kslots = n_keys;
+  if (n_keys <= sms) {
+    b.parts = sms / n_keys;
+    if (b.parts > row_tiles) b.parts = row_tiles;
+  } else {
+    b.parts = 1;
+    kslots = sms;
+  }
+  kern<<<dim3(unsigned(kslots * b.parts)), G::NT, G::SMEM, st>>>(mx, b);
+  return cudaGetLastError();
+}
+
+template <int BH, int BL>
+cudaError_t launch_strided_b(int dt_out, const StridedArgs& a, cudaStream_t st) {
+  // 32-row boxes for bf16 results, 16-row boxes for fp32 (shared-memory budget)
+  return dt_out == DT_BF16 ? launch_strided_t<BH, BL, 32, __nv_bfloat16>(a, st)
+                           : launch_strided_t<BH, BL, 16, float>(a, st);
+}
+
+}  // namespace
+
+bool strided_supported(int bh, int bl, int es_in, int es_out) {
+  // the radix of L is split between two lanes (even), P = bh bl <= 256 positions per box
+  const bool known = (bh == 7 && bl == 16) || (bh == 8 && bl == 8) || (bh == 4 && bl == 16) || (bh == 16 && bl == 4);
+  return known && es_in == 2 && (es_out == 2 || es_out == 4);
+}
+
+cudaError_t launch_bfly_strided(int bh, int bl, int dt_in, int dt_out, const StridedArgs& a, cudaStream_t st) {
+  if (dt_in != DT_BF16) return cudaErrorInvalidValue;
+  if (bh == 7 && bl == 16) return launch_strided_b<7, 16>(dt_out, a, st);
+  if (bh == 8 && bl == 8) return launch_strided_b<8, 8>(dt_out, a, st);
+  if (bh == 4 && bl == 16) return launch_strided_b<4, 16>(dt_out, a, st);
+  if (bh == 16 && bl == 4) return launch_strided_b<16, 4>(dt_out, a, st);
+  return cudaErrorInvalidValue;
+}
+
+cudaError_t wait_timeouts_strided(unsigned long long* count, bool reset) {
+  unsigned int v = 0;
+  cudaError_t e = cudaMemcpyFromSymbol(&v, g_wait_timeouts_strided, sizeof v);
+  if (e != cudaSuccess) return e;
+  *count += v;
+  if (reset && v != 0) {
+    const unsigned int zero = 0;
+    e = cudaMemcpyToSymbol(g_wait_timeouts_strided, &zero, sizeof zero);
+  }
+  return e;
+}
+
+}  // namespace hit

@@ -492,7 +492,7 @@ EncodeTiled encode_fn() {
 
 // bf16 (or fp32) tensor map, dims / strides in elements (dim 0 contiguous), 128-byte swizzle.
 bool make_map(CUtensorMap* m, const void* base, int rank, const int64_t* dims, const int64_t* strides_el,
-              const uint32_t* box, int esize = 2) {
+              const uint32_t* box, int esize = 2, bool swizzle = true) {
   EncodeTiled f = encode_fn();
   if (f == nullptr) return false;
   cuuint64_t gd[5], gs[4];
@@ -505,7 +505,8 @@ bool make_map(CUtensorMap* m, const void* base, int rank, const int64_t* dims, c
   }
   const CUtensorMapDataType dt = esize == 4 ? CU_TENSOR_MAP_DATA_TYPE_FLOAT32 : CU_TENSOR_MAP_DATA_TYPE_BFLOAT16;
   return f(m, dt, cuuint32_t(rank), const_cast<void*>(base), gd, gs, bd, es,
-           CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+           CU_TENSOR_MAP_INTERLEAVE_NONE, swizzle ? CU_TENSOR_MAP_SWIZZLE_128B : CU_TENSOR_MAP_SWIZZLE_NONE,
+           CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
            CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
@@ -623,6 +624,11 @@ cudaError_t launch_bfly_tc(const TcPassArgs& args, const void* x, int64_t ldx, c
                             : launch_tc<0, __nv_bfloat16>(mx, mm, my, a, smem, st);
   return dt_out == DT_F32 ? launch_tc<1, float>(mx, mm, my, a, smem, st)
                           : launch_tc<1, __nv_bfloat16>(mx, mm, my, a, smem, st);
+}
+
+bool make_tensor_map(CUtensorMap* m, const void* base, int rank, const int64_t* dims, const int64_t* strides_el,
+                     const uint32_t* box, int esize, bool swizzle) {
+  return make_map(m, base, rank, dims, strides_el, box, esize, swizzle);
 }
 
 cudaError_t wait_timeouts_tc(unsigned long long* count, bool reset) {

@@ -1,6 +1,7 @@
 // Internal launcher interface between the C ABI (api.cu) and the kernel
 // translation units.  Host-side C++ only; no torch types anywhere.
 #pragma once
+#include <cuda.h>
 #include <cuda_bf16.h>
 #include <cuda_runtime.h>
 #include <stddef.h>
@@ -153,5 +154,31 @@ cudaError_t launch_bfly_compose(const TcComposeArgs& a, int64_t n_windows, __nv_
 cudaError_t launch_bfly_tc(const TcPassArgs& a, const void* x, int64_t ldx, const __nv_bfloat16* mats, int dt_out,
                            cudaStream_t st);
 cudaError_t wait_timeouts_tc(unsigned long long* count, bool reset);
+// Tiled TMA tensor map (bf16 for esize 2, fp32 for 4), dims and strides in
+// elements with dim 0 contiguous, 128-byte swizzle (or a dense box without);
+// false if the driver rejects it.
+bool make_tensor_map(CUtensorMap* m, const void* base, int rank, const int64_t* dims, const int64_t* strides_el,
+                     const uint32_t* box, int esize, bool swizzle);
+
+// Two adjacent digits H (radix bh) and L (radix bl) along rows at a stride s
+// (bfly_strided.cu): positions hi * P * s + (iH * bl + iL) * s + lo.
+struct StridedArgs {
+  const void* x = nullptr;
+  void* y = nullptr;
+  int64_t ldx = 0, ldy = 0, rows = 0;
+  int64_t s = 8;        // stride of digit L (a multiple of 8)
+  int64_t n_hi = 1;     // L / (P s)
+  const float* blocks_h = nullptr;  // stage on H: [groups, bh, bh]
+  const float* blocks_l = nullptr;  // stage on L: [groups, bl, bl]
+  int shared_h = 0, shared_l = 0;   // one block for every group
+  int transpose = 0;                // transposed blocks
+  int h_first = 1;                  // stage on H applied before the stage on L
+  int64_t parts = 1;                // CTAs per key (row ranges), set by the launcher
+};
+// Whether (bh, bl) has a kernel for these element sizes, strides (elements)
+// and 16-byte aligned bases.
+bool strided_supported(int bh, int bl, int es_in, int es_out);
+cudaError_t wait_timeouts_strided(unsigned long long* count, bool reset);
+cudaError_t launch_bfly_strided(int bh, int bl, int dt_in, int dt_out, const StridedArgs& a, cudaStream_t st);
 
 }  // namespace hit

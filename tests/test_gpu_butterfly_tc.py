@@ -40,7 +40,7 @@ def test_rows(radices, transpose, out_dtype):
     assert_close(host(y), ref, torch.bfloat16, f"rows {radices} T={transpose}")
 
 
-@pytest.mark.parametrize("radices", [(7, 16, 16, 8), (4, 16, 8), (2, 16, 8, 8), (8, 8, 16), (16, 8, 16)])
+@pytest.mark.parametrize("radices", [(7, 16, 16, 8), (4, 16, 8), (2, 16, 8, 8), (8, 8, 16), (16, 8, 16), (16, 4, 8)])
 @pytest.mark.parametrize("transpose", [False, True])
 @pytest.mark.parametrize("out_dtype", [torch.bfloat16, torch.float32])
 def test_rows_strided_windows(radices, transpose, out_dtype):
