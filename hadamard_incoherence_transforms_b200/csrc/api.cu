@@ -827,7 +827,9 @@ int butterfly_apply_tc(const void* x, void* y, int64_t rows, int64_t n, int64_t 
       a.N = p.Pw;
       a.m_halves = 1;
     } else {
-      a.N = 64;
+      // 128-column data tiles where the shared-memory ring still holds
+      // several of them next to the window matrix (K = 128), 64 otherwise
+      a.N = p.Pw == 128 ? 128 : 64;
       a.m_halves = p.Pw / 128;
     }
     a.y = dst;

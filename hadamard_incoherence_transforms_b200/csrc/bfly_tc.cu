@@ -84,10 +84,25 @@ __global__ void __launch_bounds__(256) k_bfly_compose(const TcComposeArgs a, __n
       float acc[kComposeCols];
 #pragma unroll
       for (int j = 0; j < kComposeCols; ++j) acc[j] = 0.0f;
-      for (int k = 0; k < b; ++k) {
-        const float mk = st.transpose ? __ldg(blk + k * b + dig) : __ldg(blk + dig * b + k);
+      if (b <= 16) {
+        // the block row's coefficients are all loaded before the first use
+        float mk[16];
 #pragma unroll
-        for (int j = 0; j < kComposeCols; ++j) acc[j] = fmaf(mk, v[j * Pw + q0 + k * sw], acc[j]);
+        for (int k = 0; k < 16; ++k)
+          mk[k] = k < b ? (st.transpose ? __ldg(blk + k * b + dig) : __ldg(blk + dig * b + k)) : 0.0f;
+#pragma unroll
+        for (int k = 0; k < 16; ++k) {
+          if (k < b) {
+#pragma unroll
+            for (int j = 0; j < kComposeCols; ++j) acc[j] = fmaf(mk[k], v[j * Pw + q0 + k * sw], acc[j]);
+          }
+        }
+      } else {
+        for (int k = 0; k < b; ++k) {
+          const float mk = st.transpose ? __ldg(blk + k * b + dig) : __ldg(blk + dig * b + k);
+#pragma unroll
+          for (int j = 0; j < kComposeCols; ++j) acc[j] = fmaf(mk, v[j * Pw + q0 + k * sw], acc[j]);
+        }
       }
 #pragma unroll
       for (int j = 0; j < kComposeCols; ++j) u[j * Pw + q] = acc[j];
@@ -222,9 +237,16 @@ __global__ void __launch_bounds__(192, 1) k_bfly_tc(const __grid_constant__ CUte
   TcBars* bars = reinterpret_cast<TcBars*>(sout + 2 * size_t(a.bytes_out));
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
 
-  // contiguous tile range of this CTA
-  const int64_t T = a.tiles, G = gridDim.x;
-  const int64_t t_begin = blockIdx.x * T / G, t_end = (blockIdx.x + 1) * T / G;
+  // contiguous tile range of this CTA.  A column pass whose window spans two
+  // 128-row halves gives the halves to neighbouring CTAs (half = block index
+  // mod m_halves) that walk the same (window, column tile) sequence in step,
+  // so each data tile is read from DRAM once and from L2 by the other half.
+  const bool split = COLS == 1 && a.m_halves > 1;
+  const int mh = split ? int(blockIdx.x % unsigned(a.m_halves)) : 0;
+  const int64_t T = split ? a.tiles / a.m_halves : a.tiles;
+  const int64_t G = split ? int64_t(gridDim.x / unsigned(a.m_halves)) : int64_t(gridDim.x);
+  const int64_t bidx = split ? int64_t(blockIdx.x / unsigned(a.m_halves)) : int64_t(blockIdx.x);
+  const int64_t t_begin = bidx < G ? bidx * T / G : T, t_end = bidx < G ? (bidx + 1) * T / G : T;
 
   if (threadIdx.x == 0) {
     for (int s = 0; s < NS; ++s) {
@@ -261,6 +283,10 @@ __global__ void __launch_bounds__(192, 1) k_bfly_tc(const __grid_constant__ CUte
       w = key;
       half = 0;
       t0 = r * 128;
+    } else if (split) {
+      w = key;
+      half = mh;
+      t0 = r * N;
     } else {
       w = key / a.m_halves;
       half = int(key % a.m_halves);
@@ -547,6 +573,8 @@ cudaError_t launch_tc(const CUtensorMap& mx, const CUtensorMap& mm, const CUtens
   per_sm = per_sm < by_tmem ? per_sm : by_tmem;
   int64_t grid = int64_t(sms) * per_sm;
   grid = grid < a.tiles ? grid : a.tiles;
+  // column passes over two-half windows pair their CTAs (see the kernel)
+  if (COLS == 1 && a.m_halves > 1) grid -= grid % a.m_halves;
   kern<<<dim3(unsigned(grid)), 192, smem, st>>>(mx, mm, my, a);
   return cudaGetLastError();
 }
