@@ -172,7 +172,12 @@ def source_digest(sources) -> str:
 # ----------------------------------------------------------------------------
 class Workload:
     """name, algorithmic bytes and rows per step, a step(i) launching the GPU
-    hot path on rotation set i, host-buffer e2e step, and an oracle sample."""
+    hot path on rotation set i, host-buffer e2e step, and an oracle sample.
+    `dtype` is the arithmetic type of the path (fp32 registers for the SIMT
+    kernels whatever the storage type; bf16 operands with fp32 accumulation
+    on the tensor cores)."""
+
+    dtype = "f32"
 
 
 def _quant_parity(codes_rows, scales_rows, ref, bits, n) -> dict:
@@ -513,11 +518,13 @@ def two_sided_butterfly(dev, l2_bytes, host_only=False, **_):
     w.desc = ("bf16 4096x14336: R_in (7,16,16,8) along rows then R_out (16,16,16) along columns, "
               "tensor-core window products (bf16 operands, fp32 accumulation), bf16 between passes")
     w.io = "bf16 in; bf16 out"
+    w.dtype = "bf16"
     w.bytes = rows * n * 4
     w.h2d = w.d2h = rows * n * 2
-    # per side: one compose + one tcgen05 launch per pass, two passes per side
-    w.kernels_per_step = 8
-    w.kernel_key = "k_bfly_tc"
+    # R_in: strided two-digit pass, compose + tcgen05 row pass; R_out: two
+    # compose + tcgen05 column passes
+    w.kernels_per_step = 7
+    w.kernel_key = "k_bfly_strided"
 
     def oracle(r0, r1):
         from oracle import butterfly as ob
@@ -842,7 +849,7 @@ def run_gpu(args, world, rank, local):
     line = {
         "metric": METRIC, "value": value, "unit": "GB/s", "n_gpus": world, "steps": args.steps,
         "warmup": args.warmup, "ms_per_step": ms_step, "higher_is_better": True, "scaling": "weak",
-        "vs_baseline": None, "dtype": "f32", "data": "synthetic",
+        "vs_baseline": None, "dtype": w.dtype, "data": "synthetic",
         "config": {"workload": w.desc, "io": w.io, "rows": w.rows, "n": w.n,
                    "l2": f"rotating {w.rotation} input/output sets ({w.rotation * w.bytes / 1e6:.0f} MB) vs L2 {l2 / 1e6:.0f} MB",
                    "parallelism": f"replicas x{world}"},

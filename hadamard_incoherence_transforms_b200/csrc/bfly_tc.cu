@@ -45,22 +45,21 @@ namespace {
 // applied to the unit vector at position p, computed in fp32 in shared memory
 // (CC columns per CTA, ping-pong buffers).
 // ---------------------------------------------------------------------------
-constexpr int kComposeCols = 16;
-
 __device__ __forceinline__ uint32_t fdiv_u32(uint32_t n, const FastDiv& f) {
   return (__umulhi(n, f.mul) + n) >> f.shr;
 }
 
+template <int CC>
 __global__ void __launch_bounds__(256) k_bfly_compose(const TcComposeArgs a, __nv_bfloat16* __restrict__ mats) {
-  extern __shared__ float cbuf[];  // [2][kComposeCols][Pw]
+  extern __shared__ float cbuf[];  // [2][CC][Pw]
   const int Pw = a.Pw;
   const uint32_t w = blockIdx.x;
-  const int j0 = blockIdx.y * kComposeCols;
+  const int j0 = blockIdx.y * CC;
   float* v = cbuf;
-  float* u = cbuf + kComposeCols * Pw;
+  float* u = cbuf + CC * Pw;
   const uint32_t step = uint32_t(a.step);
   const uint32_t base = (w / step) * uint32_t(Pw) * step + (w % step);
-  for (int i = threadIdx.x; i < kComposeCols * Pw; i += blockDim.x) {
+  for (int i = threadIdx.x; i < CC * Pw; i += blockDim.x) {
     const int j = i / Pw, q = i - j * Pw;
     v[i] = (q == j0 + j) ? 1.0f : 0.0f;
   }
@@ -71,7 +70,7 @@ __global__ void __launch_bounds__(256) k_bfly_compose(const TcComposeArgs a, __n
     const int b = st.b;
     const int sw = int(S / step);  // the digit stride in window positions
     // every column of the chunk shares the position q: the block and the digit
-    // are found once per position, then applied to the kComposeCols columns
+    // are found once per position, then applied to the CC columns
     for (int q = threadIdx.x; q < Pw; q += blockDim.x) {
       const uint32_t g = base + uint32_t(q) * step;  // global position (< 2^31)
       const uint32_t q1 = fdiv_u32(g, st.div_s);     // g / S
@@ -81,9 +80,9 @@ __global__ void __launch_bounds__(256) k_bfly_compose(const TcComposeArgs a, __n
       const uint64_t c = st.shared_block ? 0 : uint64_t(hi) * S + lo;
       const float* blk = st.blocks + c * uint64_t(b) * uint64_t(b);
       const int q0 = q - dig * sw;
-      float acc[kComposeCols];
+      float acc[CC];
 #pragma unroll
-      for (int j = 0; j < kComposeCols; ++j) acc[j] = 0.0f;
+      for (int j = 0; j < CC; ++j) acc[j] = 0.0f;
       if (b <= 16) {
         // the block row's coefficients are all loaded before the first use
         float mk[16];
@@ -94,29 +93,40 @@ __global__ void __launch_bounds__(256) k_bfly_compose(const TcComposeArgs a, __n
         for (int k = 0; k < 16; ++k) {
           if (k < b) {
 #pragma unroll
-            for (int j = 0; j < kComposeCols; ++j) acc[j] = fmaf(mk[k], v[j * Pw + q0 + k * sw], acc[j]);
+            for (int j = 0; j < CC; ++j) acc[j] = fmaf(mk[k], v[j * Pw + q0 + k * sw], acc[j]);
           }
         }
       } else {
         for (int k = 0; k < b; ++k) {
           const float mk = st.transpose ? __ldg(blk + k * b + dig) : __ldg(blk + dig * b + k);
 #pragma unroll
-          for (int j = 0; j < kComposeCols; ++j) acc[j] = fmaf(mk, v[j * Pw + q0 + k * sw], acc[j]);
+          for (int j = 0; j < CC; ++j) acc[j] = fmaf(mk, v[j * Pw + q0 + k * sw], acc[j]);
         }
       }
 #pragma unroll
-      for (int j = 0; j < kComposeCols; ++j) u[j * Pw + q] = acc[j];
+      for (int j = 0; j < CC; ++j) u[j * Pw + q] = acc[j];
     }
     __syncthreads();
     float* tmp = v;
     v = u;
     u = tmp;
   }
-  // row q, column j0 + j of the window's matrix
+  // row q, columns j0 .. j0 + CC - 1 of the window's matrix: one thread per
+  // row reads its column of the buffer (consecutive lanes, consecutive words)
+  // and writes the CC values as 16-byte pieces
   __nv_bfloat16* out = mats + uint64_t(w) * uint64_t(Pw) * Pw;
-  for (int i = threadIdx.x; i < kComposeCols * Pw; i += blockDim.x) {
-    const int q = i / kComposeCols, j = i - q * kComposeCols;
-    out[uint64_t(q) * Pw + j0 + j] = __float2bfloat16_rn(v[j * Pw + q]);
+  for (int q = threadIdx.x; q < Pw; q += blockDim.x) {
+    uint4* dst = reinterpret_cast<uint4*>(out + uint64_t(q) * Pw + j0);
+#pragma unroll
+    for (int c = 0; c < CC / 8; ++c) {
+      uint32_t p[4];
+#pragma unroll
+      for (int e = 0; e < 4; ++e) {
+        const int j = 8 * c + 2 * e;
+        p[e] = f32_to_bf16x2(v[j * Pw + q], v[(j + 1) * Pw + q]);
+      }
+      dst[c] = make_uint4(p[0], p[1], p[2], p[3]);
+    }
   }
 }
 
@@ -582,12 +592,24 @@ cudaError_t launch_tc(const CUtensorMap& mx, const CUtensorMap& mm, const CUtens
 }  // namespace
 
 cudaError_t launch_bfly_compose(const TcComposeArgs& a, int64_t n_windows, __nv_bfloat16* mats, cudaStream_t st) {
-  static std::atomic<unsigned long long> done{0};
-  const size_t smem = size_t(2) * kComposeCols * a.Pw * sizeof(float);
-  cudaError_t e = smem_attr_once(k_bfly_compose, smem, done);
-  if (e != cudaSuccess) return e;
+  // 64 columns per CTA up to 128-position windows, 32 for 256 (64 KB of
+  // buffers either way); 16 for windows narrower than 64
+  static std::atomic<unsigned long long> done16{0}, done32{0}, done64{0};
   const int threads = a.Pw >= 256 ? 256 : ((a.Pw + 31) / 32) * 32;
-  k_bfly_compose<<<dim3(unsigned(n_windows), unsigned(a.Pw / kComposeCols)), threads, smem, st>>>(a, mats);
+  cudaError_t e;
+  if (a.Pw % 64 == 0 && a.Pw <= 128) {
+    const size_t smem = size_t(2) * 64 * a.Pw * sizeof(float);
+    if ((e = smem_attr_once(k_bfly_compose<64>, smem, done64)) != cudaSuccess) return e;
+    k_bfly_compose<64><<<dim3(unsigned(n_windows), unsigned(a.Pw / 64)), threads, smem, st>>>(a, mats);
+  } else if (a.Pw % 32 == 0) {
+    const size_t smem = size_t(2) * 32 * a.Pw * sizeof(float);
+    if ((e = smem_attr_once(k_bfly_compose<32>, smem, done32)) != cudaSuccess) return e;
+    k_bfly_compose<32><<<dim3(unsigned(n_windows), unsigned(a.Pw / 32)), threads, smem, st>>>(a, mats);
+  } else {
+    const size_t smem = size_t(2) * 16 * a.Pw * sizeof(float);
+    if ((e = smem_attr_once(k_bfly_compose<16>, smem, done16)) != cudaSuccess) return e;
+    k_bfly_compose<16><<<dim3(unsigned(n_windows), unsigned(a.Pw / 16)), threads, smem, st>>>(a, mats);
+  }
   return cudaGetLastError();
 }
 

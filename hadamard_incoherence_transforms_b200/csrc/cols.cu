@@ -321,6 +321,7 @@ __global__ void __launch_bounds__(ClusterSmem<Tin>::THREADS) k_cols_cluster(cons
       for (int c = 0; c < CL; ++c)
         post_m |= uint32_t(a.post_signs[int64_t(c) * 1024 + crank * SHARE + tr + 32 * u] < 0) << (u * CL + c);
   }
+  bool pending = false;  // this thread arrived on the cluster barrier after a strip's reads
   for (; strip < strips; strip += clusters) {
     cp_async_wait_all();
     __syncthreads();  // every thread's copies of this strip have landed
@@ -347,6 +348,8 @@ __global__ void __launch_bounds__(ClusterSmem<Tin>::THREADS) k_cols_cluster(cons
     __syncthreads();  // the staging rows are free: start streaming the next strip
     if (strip + clusters < strips) prefetch(strip + clusters);
     reg_stages<128, 2, 7>(x);  // row bits 5..9
+    // the cluster's phase-3 reads of this CTA's previous block are done
+    if (pending) asm volatile("barrier.cluster.wait.aligned;" ::: "memory");
 #pragma unroll
     for (int k = 0; k < 32; ++k)
       cs_smem[cs_idx<kQuads>(tr + 32 * k, q)] = make_float4(x[4 * k], x[4 * k + 1], x[4 * k + 2], x[4 * k + 3]);
@@ -365,17 +368,32 @@ __global__ void __launch_bounds__(ClusterSmem<Tin>::THREADS) k_cols_cluster(cons
     cluster.sync();  // all blocks of the strip are in shared memory
     // phase 3: this CTA combines rows (c', row_low) for row_low in its share
     Tout* dst = static_cast<Tout*>(a.y) + strip * 4 * kQuads + 4 * q;
+    // every remote read of the strip is issued before the first is used
+    float vall[SHARE / 32][4 * CL];
 #pragma unroll
     for (int u = 0; u < SHARE / 32; ++u) {
       const int row_low = crank * SHARE + tr + 32 * u;
-      float v[4 * CL];
 #pragma unroll
       for (int c = 0; c < CL; ++c) {
         const float4* rem = cluster.map_shared_rank(cs_smem, c);
         const float4 w = rem[cs_idx<kQuads>(row_low, q)];
-        v[4 * c] = w.x; v[4 * c + 1] = w.y; v[4 * c + 2] = w.z; v[4 * c + 3] = w.w;
+        vall[u][4 * c] = w.x; vall[u][4 * c + 1] = w.y; vall[u][4 * c + 2] = w.z; vall[u][4 * c + 3] = w.w;
       }
-      if constexpr (CL > 1) reg_stages<4 * CL, 2, 2 + (CL == 2 ? 1 : (CL == 4 ? 2 : 3))>(v);
+    }
+    // the remaining stages consume every value read (so the reads have
+    // completed) before this CTA releases its hold on the cluster's blocks
+    // with a relaxed arrive; the matching wait comes before the next strip's
+    // first write to shared memory (or at exit)
+    if constexpr (CL > 1) {
+#pragma unroll
+      for (int u = 0; u < SHARE / 32; ++u) reg_stages<4 * CL, 2, 2 + (CL == 2 ? 1 : (CL == 4 ? 2 : 3))>(vall[u]);
+    }
+    asm volatile("barrier.cluster.arrive.relaxed.aligned;" ::: "memory");
+    pending = true;
+#pragma unroll
+    for (int u = 0; u < SHARE / 32; ++u) {
+      const int row_low = crank * SHARE + tr + 32 * u;
+      const float(&v)[4 * CL] = vall[u];
 #pragma unroll
       for (int c = 0; c < CL; ++c) {
         const int64_t r = int64_t(c) * 1024 + row_low;
@@ -388,8 +406,9 @@ __global__ void __launch_bounds__(ClusterSmem<Tin>::THREADS) k_cols_cluster(cons
         }
       }
     }
-    cluster.sync();  // no CTA rewrites its block while others still read it
   }
+  // no CTA leaves while others may still read its block
+  if (pending) asm volatile("barrier.cluster.wait.aligned;" ::: "memory");
   cp_async_wait_all();  // nothing in flight into this CTA's shared memory at exit
 }
 
