@@ -256,34 +256,95 @@ __device__ __forceinline__ void dequant_rowB(float (&x)[Geom<LOGN>::E], const Ro
 
 // Sparse adapter, forward: F_r = scatter-add of (values * scale) at cols into
 // a zeroed row buffer, then read back in layout B.
+// Up to kScatterPre entries per thread are held in registers, loaded before
+// the row buffer is cleared so that their latency overlaps the clearing.
+constexpr int kScatterPre = 4;
 template <int LOGN>
-__device__ __forceinline__ void scatter_rowB(float (&x)[Geom<LOGN>::E], const RowArgs& a, int64_t row, int tau,
-                                             int team, float4* buf) {
+__device__ __forceinline__ void scatter_load(int (&cols)[kScatterPre], float (&vals)[kScatterPre], const RowArgs& a,
+                                             int64_t row, int tau) {
   using G = Geom<LOGN>;
+  const int64_t base = row * a.nnz;
+#pragma unroll
+  for (int j = 0; j < kScatterPre; ++j) {
+    const int k = tau + j * G::T;
+    cols[j] = -1;
+    vals[j] = 0.0f;
+    if (k < a.nnz) {
+      cols[j] = __ldg(a.sp_cols + base + k);
+      vals[j] = __ldg(a.sp_values + base + k);
+    }
+  }
+}
+// Clear the row buffer, add the row's entries (held in registers when `fast`,
+// else read here) and read the row back in layout B.
+template <int LOGN>
+__device__ __forceinline__ void scatter_apply(float (&x)[Geom<LOGN>::E], const RowArgs& a, int64_t row, int tau,
+                                              int team, float4* buf, bool fast, const int (&cols)[kScatterPre],
+                                              const float (&vals)[kScatterPre]) {
+  using G = Geom<LOGN>;
+  float* bf = reinterpret_cast<float*>(buf);
 #pragma unroll
   for (int m = 0; m < G::E / 4; ++m) buf[swz<G::LQ>((G::E / 4) * tau + m)] = make_float4(0.f, 0.f, 0.f, 0.f);
   team_sync<G::T>(team);
-  float* bf = reinterpret_cast<float*>(buf);
-  const int64_t base = row * a.nnz;
-  for (int k = tau; k < a.nnz; k += G::T) {
-    const int col = __ldg(a.sp_cols + base + k);
-    if (static_cast<unsigned>(col) < static_cast<unsigned>(G::N))
-      atomicAdd(bf + smem_elem<LOGN>(col), __ldg(a.sp_values + base + k) * a.sp_scale);
+  if (fast) {
+#pragma unroll
+    for (int j = 0; j < kScatterPre; ++j)
+      if (static_cast<unsigned>(cols[j]) < static_cast<unsigned>(G::N))
+        atomicAdd(bf + smem_elem<LOGN>(cols[j]), vals[j] * a.sp_scale);
+  } else {
+    const int64_t base = row * a.nnz;
+    for (int k = tau; k < a.nnz; k += G::T) {
+      const int col = __ldg(a.sp_cols + base + k);
+      if (static_cast<unsigned>(col) < static_cast<unsigned>(G::N))
+        atomicAdd(bf + smem_elem<LOGN>(col), __ldg(a.sp_values + base + k) * a.sp_scale);
+    }
   }
   team_sync<G::T>(team);
   smem_get_B<LOGN>(buf, x, tau);
 }
+template <int LOGN>
+__device__ __forceinline__ void scatter_rowB(float (&x)[Geom<LOGN>::E], const RowArgs& a, int64_t row, int tau,
+                                             int team, float4* buf) {
+  using G = Geom<LOGN>;
+  int cols[kScatterPre];
+  float vals[kScatterPre];
+  const bool fast = a.nnz <= kScatterPre * G::T;
+  if (fast) scatter_load<LOGN>(cols, vals, a, row, tau);
+  scatter_apply<LOGN>(x, a, row, tau, team, buf, fast, cols, vals);
+}
 
 // Sparse adapter, backward: out[k] = (row transform * scale)[cols[k]].
+// Up to kGatherPre column indices per thread are read before the row (see
+// k_rows_a2b), so their latency overlaps the row's load and transform.
+constexpr int kGatherPre = 4;
+template <int LOGN>
+__device__ __forceinline__ void gather_cols_pre(int (&cols)[kGatherPre], const RowArgs& a, int64_t row, int tau) {
+  using G = Geom<LOGN>;
+  const int64_t base = row * a.nnz;
+#pragma unroll
+  for (int j = 0; j < kGatherPre; ++j) {
+    const int k = tau + j * G::T;
+    cols[j] = k < a.nnz ? __ldg(a.sp_cols + base + k) : -1;
+  }
+}
 template <int LOGN>
 __device__ __forceinline__ void gather_rowB(const float (&x)[Geom<LOGN>::E], const RowArgs& a, int64_t row, int tau,
-                                            int team, float4* buf) {
+                                            int team, float4* buf, const int (&cols)[kGatherPre]) {
   using G = Geom<LOGN>;
   smem_put_B<LOGN>(buf, x, tau);
   team_sync<G::T>(team);
   const float* bf = reinterpret_cast<const float*>(buf);
   const int64_t base = row * a.nnz;
-  for (int k = tau; k < a.nnz; k += G::T) {
+#pragma unroll
+  for (int j = 0; j < kGatherPre; ++j) {
+    const int k = tau + j * G::T;
+    if (k < a.nnz) {
+      float v = 0.0f;
+      if (static_cast<unsigned>(cols[j]) < static_cast<unsigned>(G::N)) v = bf[smem_elem<LOGN>(cols[j])] * a.sp_scale;
+      a.sp_out[base + k] = v;
+    }
+  }
+  for (int k = tau + kGatherPre * G::T; k < a.nnz; k += G::T) {
     const int col = __ldg(a.sp_cols + base + k);
     float v = 0.0f;
     if (static_cast<unsigned>(col) < static_cast<unsigned>(G::N)) v = bf[smem_elem<LOGN>(col)] * a.sp_scale;
@@ -307,6 +368,8 @@ __global__ void __launch_bounds__(Geom<LOGN>::NT, Geom<LOGN>::MINB) k_rows_a2b(c
   float4* buf = smem4 + size_t(team) * (G::N / 4);
 
   float x[G::E];
+  int gcols[kGatherPre];
+  if constexpr (EPI == EPI_GATHER) gather_cols_pre<LOGN>(gcols, a, row, tau);
   load_rowA<LOGN, Tin>(x, static_cast<const Tin*>(a.x) + row * a.ldx, tau, a.pre_signs);
   reg_stages<G::E, 0, G::LOGE>(x);
   if constexpr (G::T > 1) {
@@ -322,7 +385,7 @@ __global__ void __launch_bounds__(Geom<LOGN>::NT, Geom<LOGN>::MINB) k_rows_a2b(c
   } else if constexpr (EPI == EPI_QUANT) {
     quant_rowB<LOGN, BITS>(x, a, row, tau);
   } else {
-    gather_rowB<LOGN>(x, a, row, tau, team, buf);
+    gather_rowB<LOGN>(x, a, row, tau, team, buf, gcols);
   }
 }
 
