@@ -57,6 +57,22 @@ def test_rows_strided_windows(radices, transpose, out_dtype):
     assert_close(host(y), ref, torch.bfloat16, f"strided rows {radices} T={transpose}")
 
 
+@pytest.mark.parametrize("rows,radices", [(40, (7, 16, 8, 8, 8, 2, 2)), (5, (7, 16, 16, 8)), (33, (4, 16, 8, 4, 8))])
+@pytest.mark.parametrize("transpose", [False, True])
+def test_rows_strided_shapes(rows, radices, transpose):
+    """Strided two-digit runs with more (lo group, hi) keys than SMs (the
+    (7, 16) run at stride 2048: 256 keys), fewer rows than one 32-row tile,
+    and a run whose boxes reach past the last hi block; fp32 results."""
+    d = int(np.prod(radices))
+    blocks = blocks_for(radices, seed=d + 11)
+    bits, xf = bf16_input((rows, d), d + 11)
+    y = hit.butterfly_apply_tc(to_gpu_bf16(bits), radices, [to_gpu_f32(b) for b in blocks], axis=1,
+                               transpose=transpose, out_dtype=torch.float32)
+    torch.cuda.synchronize()
+    ref = ob.apply_stages(xf, radices, blocks, transpose)
+    assert_close(host(y), ref, torch.bfloat16, f"strided rows {radices} x {rows} T={transpose}")
+
+
 @pytest.mark.parametrize("radices", [(16, 16, 16), (8, 16), (2, 4, 16), (16, 8, 2), (4, 32, 2)])
 @pytest.mark.parametrize("transpose", [False, True])
 def test_columns(radices, transpose):
