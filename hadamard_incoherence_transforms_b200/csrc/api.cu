@@ -827,9 +827,10 @@ int butterfly_apply_tc(const void* x, void* y, int64_t rows, int64_t n, int64_t 
       a.N = p.Pw;
       a.m_halves = 1;
     } else {
-      // 128-column data tiles where the shared-memory ring still holds
-      // several of them next to the window matrix (K = 128), 64 otherwise
-      a.N = p.Pw == 128 ? 128 : 64;
+      // 128-column data tiles (for K = 256 the output is staged in one
+      // buffer so that two data stages fit next to the half window matrix);
+      // 64 columns for K = 256 with fp32 results (a 64 KB staged tile)
+      a.N = (p.Pw == 256 && dt_dst == HIT_F32) ? 64 : 128;
       a.m_halves = p.Pw / 128;
     }
     a.y = dst;

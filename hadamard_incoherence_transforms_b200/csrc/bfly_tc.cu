@@ -244,7 +244,7 @@ __global__ void __launch_bounds__(192, 1) k_bfly_tc(const __grid_constant__ CUte
   uint8_t* smat = smem;                                   // window matrix (A for COLS 1, B for COLS 0)
   uint8_t* sdat = smem + size_t(a.bytes_mat);             // NS data stages
   uint8_t* sout = sdat + size_t(NS) * a.bytes_stage;       // two output tiles (TMA store sources)
-  TcBars* bars = reinterpret_cast<TcBars*>(sout + 2 * size_t(a.bytes_out));
+  TcBars* bars = reinterpret_cast<TcBars*>(sout + size_t(a.out_bufs) * a.bytes_out);
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
 
   // contiguous tile range of this CTA.  A column pass whose window spans two
@@ -426,14 +426,18 @@ __global__ void __launch_bounds__(192, 1) k_bfly_tc(const __grid_constant__ CUte
         if (lane == 0) atomicAdd(&g_wait_timeouts_tc, 1u);
       }
       // the staging buffer of tile i - 2 must have been read by its stores
-      if (threadIdx.x == 0 && i >= 2) asm volatile("cp.async.bulk.wait_group.read 1;" ::: "memory");
+      // (with one staging buffer: the previous tile's)
+      if (threadIdx.x == 0 && i >= a.out_bufs) {
+        if (a.out_bufs == 2) asm volatile("cp.async.bulk.wait_group.read 1;" ::: "memory");
+        else asm volatile("cp.async.bulk.wait_group.read 0;" ::: "memory");
+      }
       // one decision for the four warps (they meet at named barriers below)
       if (!bar_and_128(ok)) {
         *abort = 1;
         break;
       }
       asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory");
-      uint8_t* ob = sout + size_t(ab) * a.bytes_out;
+      uint8_t* ob = sout + size_t(a.out_bufs == 2 ? ab : 0) * a.bytes_out;
       for (int c = 0; c < N / 32; ++c) {
         uint32_t v[32];
         tmem_ld32(tmem + (uint32_t(32 * warp) << 16) + uint32_t(ab * N + 32 * c), v);
@@ -660,11 +664,17 @@ cudaError_t launch_bfly_tc(const TcPassArgs& args, const void* x, int64_t ldx, c
   a.bytes_out = 128 * a.N * eo;
   a.tmem_cols = 2 * a.N <= 64 ? 64 : (2 * a.N <= 128 ? 128 : (2 * a.N <= 256 ? 256 : 512));
   // one CTA per SM: the window matrix, two output tiles and as many data
-  // stages as fit (at most six)
-  const size_t fixed = 1024 + size_t(a.bytes_mat) + 2 * size_t(a.bytes_out) + 512;
+  // stages as fit (at most six); one output tile when two would leave fewer
+  // than two data stages
   const size_t whole = 226 * 1024;
-  if (fixed >= whole) return cudaErrorInvalidValue;
-  int ns = int((whole - fixed) / size_t(a.bytes_stage));
+  size_t fixed = 0;
+  int ns = 0;
+  for (int ob = 2; ob >= 1; --ob) {
+    fixed = 1024 + size_t(a.bytes_mat) + size_t(ob) * size_t(a.bytes_out) + 512;
+    ns = fixed < whole ? int((whole - fixed) / size_t(a.bytes_stage)) : 0;
+    a.out_bufs = ob;
+    if (ns >= 2) break;
+  }
   ns = ns > 6 ? 6 : ns;
   if (ns < 1) return cudaErrorInvalidValue;
   a.stages = ns;

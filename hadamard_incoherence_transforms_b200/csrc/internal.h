@@ -145,6 +145,7 @@ struct TcPassArgs {
   int n_windows = 0, m_halves = 1, tmem_cols = 0;
   int bytes_mat = 0, bytes_stage = 0;  // window matrix / one data tile in shared memory
   int bytes_out = 0;                   // one output tile staged for its TMA store
+  int out_bufs = 2;                    // output staging buffers (2: a tile's stores drain under the next)
   int stages = 1;                      // data tiles in flight per CTA
   int64_t tiles = 0, tiles_per_key = 1;  // tiles of the pass; consecutive tiles sharing a window matrix
   void* y = nullptr;
