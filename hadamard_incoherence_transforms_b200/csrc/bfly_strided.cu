@@ -19,7 +19,8 @@
 // previous one is computed.  A lane holds half of the vector (the iL of one
 // parity, h, for every iH) of two rows of one lo: the stage on H is local, the
 // stage on L takes the partner half (lane ^ 16) by shuffles, and every
-// coefficient read from shared memory feeds both rows with packed fp32 FMAs.
+// coefficient read from shared memory (bf16, eight per 16-byte read) feeds
+// both rows with packed fp32 FMAs.
 // Lane = h * 16 + rp * 8 + lo: the eight lo values of a half-warp read eight
 // different blocks laid out 4 words apart in the banks (one wavefront), and the
 // four (row, parity) pairs of a lo value read 16-byte rows in four distinct
@@ -42,31 +43,35 @@ __device__ unsigned int g_wait_timeouts_strided = 0;
 
 namespace {
 
-// Coefficients of one lo value in shared memory.  Stage on H: block iL at
-// iL BH BHP, entry (k, a) at k BHP + a = coefficient of output a from input k.
-// Stage on L: block iH at HF + iH BL BLP, entry (k, a) at k BLP + perm(a) with
-// the even outputs first, perm(a) = (a & 1) HL + a / 2, so that the outputs of
-// one parity are contiguous.  PER_LO is 4 mod 32 words: the blocks of eight lo
-// values start in eight different 4-bank groups.
+// Coefficients of one lo value in shared memory, as bf16 (the tensor-core
+// path's operand precision; every read then carries eight coefficients).
+// Stage on H: block iL at iL BH BHP, entry (k, a) at k BHP + a = coefficient
+// of output a from input k.  Stage on L: block iH at HF + iH BL BLP, entry
+// (k, a) at k BLP + perm(a) with the even outputs first, perm(a) = (a & 1) HL +
+// a / 2, so that the outputs of one parity are contiguous.  PER_LO is 8 mod 64
+// elements (16 mod 128 bytes): the blocks of eight lo values start in eight
+// different 4-bank groups.
 template <int BH, int BL>
 struct StridedBlocks {
   static constexpr int BHP = (BH + 3) / 4 * 4;
   static constexpr int BLP = (BL + 3) / 4 * 4;
   static constexpr int HL = BL / 2;
-  static constexpr int HF = BL * BH * BHP + 4;
+  static constexpr int HF0 = BL * BH * BHP;
   static constexpr int LF = BH * BL * BLP;
+  static constexpr int PAD = ((8 - (HF0 + LF) % 64) + 64) % 64;
+  static constexpr int HF = HF0 + PAD;
   static constexpr int PER_LO = HF + LF;
   static_assert(BL % 2 == 0, "the radix of L is split by parity");
-  static_assert(PER_LO % 32 == 4, "block layout must start the lo values in distinct bank groups");
+  static_assert(PER_LO % 64 == 8 && HF % 8 == 0, "block layout must start the lo values in distinct bank groups");
 };
 
 // Stage the coefficients of one stage for the eight lo values of a group.  The
 // blocks of groups run0 + d * run_stride + l (l = 0..7) are eight consecutive
 // blocks in global memory for each of the NR run digits d, so every run is one
 // contiguous stretch of 8 B^2 floats: read coalesced, eight loads in flight per
-// thread.
+// thread, rounded to bf16.
 template <int B, int BP, int NR, bool PERM, int NT>
-__device__ __forceinline__ void stage_blocks(float* s_blk, int per_lo, int ofs, const float* blocks, int64_t run0,
+__device__ __forceinline__ void stage_blocks(uint16_t* s_blk, int per_lo, int ofs, const float* blocks, int64_t run0,
                                              int64_t run_stride, bool shared, bool transpose) {
   constexpr int BB = B * B;
   constexpr int RUN = 8 * BB;
@@ -90,7 +95,7 @@ __device__ __forceinline__ void stage_blocks(float* s_blk, int per_lo, int ofs, 
         const int l = e / BB, f = e - l * BB, rr = f / B, cc = f - rr * B;  // entry (rr, cc) of block l
         const int k = transpose ? rr : cc, aa = transpose ? cc : rr;
         const int col = PERM ? (aa & 1) * (B / 2) + (aa >> 1) : aa;
-        s_blk[l * per_lo + ofs + d * B * BP + k * BP + col] = g[u];
+        s_blk[l * per_lo + ofs + d * B * BP + k * BP + col] = __bfloat16_as_ushort(__float2bfloat16_rn(g[u]));
       }
     }
   }
@@ -114,37 +119,40 @@ __device__ __forceinline__ void st_elem(uint8_t* p, float v) {
   else *reinterpret_cast<uint16_t*>(p) = __bfloat16_as_ushort(__float2bfloat16_rn(v));
 }
 
-// {o[q], o[q + 1]} += {c0, c1} * s for two rows sharing the coefficients
-__device__ __forceinline__ void fma2_rows(float c0, float c1, float s0, float s1, float& a0, float& a1, float& b0,
-                                          float& b1) {
-  fma_x2(c0, c1, s0, s0, a0, a1, a0, a1);
-  fma_x2(c0, c1, s1, s1, b0, b1, b0, b1);
-}
-
-// o_r[q] += b[q] * s_r (q < N, two rows) from 16- (or 8-) byte coefficient loads
-template <int N>
-__device__ __forceinline__ void axpy2(const float* b, float s0, float s1, float* o0, float* o1) {
-  if constexpr (N % 4 == 0 || N > 4) {
+// o_r[q] += b[q] * s[r] for the RPL rows of a lane, q < N, from the N (padded
+// to a multiple of four) consecutive bf16 coefficients at b: 16-byte reads of
+// eight coefficients (8 or 4 bytes for four or two), packed fp32 FMAs on
+// coefficient pairs.
+__device__ __forceinline__ float bf_lo(uint32_t w) { return __uint_as_float(w << 16); }
+__device__ __forceinline__ float bf_hi(uint32_t w) { return __uint_as_float(w & 0xffff0000u); }
+template <int N, int RPL>
+__device__ __forceinline__ void pair_fma(uint32_t w, int q, const float (&s)[RPL], float (&o)[RPL][N]) {
+  if (q + 1 < N) {
 #pragma unroll
-    for (int q4 = 0; q4 < (N + 3) / 4; ++q4) {
-      const float4 c = *reinterpret_cast<const float4*>(b + 4 * q4);
-      if (4 * q4 + 1 < N) {
-        fma2_rows(c.x, c.y, s0, s1, o0[4 * q4], o0[4 * q4 + 1], o1[4 * q4], o1[4 * q4 + 1]);
-      } else {
-        o0[4 * q4] = fmaf(c.x, s0, o0[4 * q4]);
-        o1[4 * q4] = fmaf(c.x, s1, o1[4 * q4]);
-      }
-      if (4 * q4 + 3 < N) {
-        fma2_rows(c.z, c.w, s0, s1, o0[4 * q4 + 2], o0[4 * q4 + 3], o1[4 * q4 + 2], o1[4 * q4 + 3]);
-      } else if (4 * q4 + 2 < N) {
-        o0[4 * q4 + 2] = fmaf(c.z, s0, o0[4 * q4 + 2]);
-        o1[4 * q4 + 2] = fmaf(c.z, s1, o1[4 * q4 + 2]);
-      }
+    for (int r = 0; r < RPL; ++r) fma_x2(bf_lo(w), bf_hi(w), s[r], s[r], o[r][q], o[r][q + 1], o[r][q], o[r][q + 1]);
+  } else if (q < N) {
+#pragma unroll
+    for (int r = 0; r < RPL; ++r) o[r][q] = fmaf(bf_lo(w), s[r], o[r][q]);
+  }
+}
+template <int N, int RPL>
+__device__ __forceinline__ void axpy_bf(const uint16_t* b, const float (&s)[RPL], float (&o)[RPL][N]) {
+  if constexpr (N > 4) {
+#pragma unroll
+    for (int c8 = 0; c8 < (N + 7) / 8; ++c8) {
+      const uint4 w = *reinterpret_cast<const uint4*>(b + 8 * c8);
+      pair_fma<N, RPL>(w.x, 8 * c8, s, o);
+      pair_fma<N, RPL>(w.y, 8 * c8 + 2, s, o);
+      pair_fma<N, RPL>(w.z, 8 * c8 + 4, s, o);
+      pair_fma<N, RPL>(w.w, 8 * c8 + 6, s, o);
     }
+  } else if constexpr (N > 2) {
+    const uint2 w = *reinterpret_cast<const uint2*>(b);
+    pair_fma<N, RPL>(w.x, 0, s, o);
+    pair_fma<N, RPL>(w.y, 2, s, o);
   } else {
-    static_assert(N == 2, "row segment of 2, 4k or more than 4 coefficients");
-    const float2 c = *reinterpret_cast<const float2*>(b);
-    fma2_rows(c.x, c.y, s0, s1, o0[0], o0[1], o1[0], o1[1]);
+    static_assert(N == 2, "row segment of 2 or more coefficients");
+    pair_fma<N, RPL>(*reinterpret_cast<const uint32_t*>(b), 0, s, o);
   }
 }
 
@@ -155,25 +163,27 @@ __device__ __forceinline__ void tma_load_3d(void* dst, const CUtensorMap* map, i
       "l"(map), "r"(c0), "r"(c1), "r"(c2), "r"(smem_u32(bar))
       : "memory");
 }
-template <int BH, int BL, int R, typename Tout>
+template <int BH, int BL, int RPL, typename Tout>
 struct StridedGeom {
   static constexpr int P = BH * BL;
-  static constexpr int NT = 8 * R;  // R / 2 row pairs x 8 lo x 2 halves
+  static constexpr int NT = 256;       // 8 warps x (2 row groups x 8 lo x 2 halves)
+  static constexpr int R = 16 * RPL;   // rows per box: RPL rows per lane
   static constexpr int IN_BYTES = R * (P + 1) * 8 * 2;
   static constexpr int OUT_BYTES = R * (P + 1) * 8 * int(sizeof(Tout));
   static constexpr int IN_OFS = 0;  // 1024-byte aligned box
   static constexpr int OUT_OFS = (IN_BYTES + 1023) / 1024 * 1024;
   static constexpr int BLK_OFS = OUT_OFS + (OUT_BYTES + 15) / 16 * 16;
-  static constexpr int BAR_OFS = BLK_OFS + 8 * StridedBlocks<BH, BL>::PER_LO * 4;
+  static constexpr int BAR_OFS = BLK_OFS + 8 * StridedBlocks<BH, BL>::PER_LO * 2;
   static constexpr int SMEM = BAR_OFS + 16 + 1024;  // + slack to align the base
 };
 
-template <int BH, int BL, int R, typename Tout>
-__global__ void __launch_bounds__(8 * R, 1)
+template <int BH, int BL, int RPL, typename Tout>
+__global__ void __launch_bounds__(256, 1)
     k_bfly_strided(const __grid_constant__ CUtensorMap map_x, const StridedArgs a) {
   using SB = StridedBlocks<BH, BL>;
-  using G = StridedGeom<BH, BL, R, Tout>;
+  using G = StridedGeom<BH, BL, RPL, Tout>;
   constexpr int P = G::P;
+  constexpr int R = G::R;
   constexpr int HL = SB::HL;
   constexpr int NV = BH * HL;  // values per lane and row
   constexpr int EO = int(sizeof(Tout));
@@ -181,12 +191,12 @@ __global__ void __launch_bounds__(8 * R, 1)
   uint8_t* sm = smem_raw + ((1024u - (smem_u32(smem_raw) & 1023u)) & 1023u);
   uint8_t* s_in = sm + G::IN_OFS;
   uint8_t* s_out = sm + G::OUT_OFS;
-  float* s_blk = reinterpret_cast<float*>(sm + G::BLK_OFS);
+  uint16_t* s_blk = reinterpret_cast<uint16_t*>(sm + G::BLK_OFS);
   uint64_t* full = reinterpret_cast<uint64_t*>(sm + G::BAR_OFS);
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int h = lane >> 4, rp = (lane >> 3) & 1, lo = lane & 7;
-  const int row0 = 4 * warp + 2 * rp;  // this lane's rows row0, row0 + 1 of the box
+  const int row0 = (2 * warp + rp) * RPL;  // this lane's rows row0 .. row0 + RPL - 1 of the box
   const int64_t S = a.s;
   const int64_t groups8 = S / 8;
   const int64_t n_keys = a.n_hi * groups8;
@@ -200,9 +210,7 @@ __global__ void __launch_bounds__(8 * R, 1)
   const int64_t ks = blockIdx.x % kslots, part = blockIdx.x / kslots;
   const int64_t rt_begin = part * row_tiles / a.parts, rt_end = (part + 1) * row_tiles / a.parts;
   if (ks >= n_keys || rt_begin >= rt_end) return;
-  const __nv_bfloat16* x = static_cast<const __nv_bfloat16*>(a.x);
   Tout* y = static_cast<Tout*>(a.y);
-  (void)x;
   if (threadIdx.x == 0) {
     mbar_init(full, 1);
     mbar_init_fence();
@@ -210,7 +218,7 @@ __global__ void __launch_bounds__(8 * R, 1)
     tma_load_3d(s_in, &map_x, int((ks % groups8) * 8), int((ks / groups8) * P), int(rt_begin * R), full);
   }
   uint32_t phase = 0;
-  const float* bl = s_blk + lo * SB::PER_LO;
+  const uint16_t* bl = s_blk + lo * SB::PER_LO;
   for (int64_t key = ks; key < n_keys; key += kslots) {
     const int64_t hi = key / groups8, lo0 = (key % groups8) * 8;
     const int64_t col0 = hi * int64_t(P) * S + lo0;  // column of (iH, iL) = (0, 0), lo = lo0
@@ -223,16 +231,15 @@ __global__ void __launch_bounds__(8 * R, 1)
     for (int64_t rt = rt_begin; rt < rt_end; ++rt) {
       const bool ok = mbar_wait(full, phase);
       phase ^= 1u;
-      // this lane's half vectors: v_r[iH * HL + j] = position iH BL + 2 j + h of row row0 + r
-      float v0[NV], v1[NV];
+      // this lane's half vectors: v[r][iH * HL + j] = position iH BL + 2 j + h of row row0 + r
+      float v[RPL][NV];
 #pragma unroll
-      for (int iH = 0; iH < BH; ++iH)
+      for (int r = 0; r < RPL; ++r)
 #pragma unroll
-        for (int j = 0; j < HL; ++j) {
-          const int p = iH * BL + 2 * j + h;
-          v0[iH * HL + j] = ld_elem<__nv_bfloat16>(s_in + box_offset<P, 2>(row0, p, lo));
-          v1[iH * HL + j] = ld_elem<__nv_bfloat16>(s_in + box_offset<P, 2>(row0 + 1, p, lo));
-        }
+        for (int iH = 0; iH < BH; ++iH)
+#pragma unroll
+          for (int j = 0; j < HL; ++j)
+            v[r][iH * HL + j] = ld_elem<__nv_bfloat16>(s_in + box_offset<P, 2>(row0 + r, iH * BL + 2 * j + h, lo));
       // every lane has read the box (and the previous tile's results have
       // left the output tile): the next box may land
       if (!__syncthreads_and(ok)) {
@@ -253,41 +260,51 @@ __global__ void __launch_bounds__(8 * R, 1)
       auto stage_h = [&]() {
 #pragma unroll
         for (int j = 0; j < HL; ++j) {
-          const float* b = bl + (2 * j + h) * BH * SB::BHP;  // block iL = 2 j + h
-          float o0[BH], o1[BH];
+          const uint16_t* b = bl + (2 * j + h) * BH * SB::BHP;  // block iL = 2 j + h
+          float o[RPL][BH];
 #pragma unroll
-          for (int q = 0; q < BH; ++q) o0[q] = o1[q] = 0.0f;
+          for (int r = 0; r < RPL; ++r)
 #pragma unroll
-          for (int k = 0; k < BH; ++k) axpy2<BH>(b + k * SB::BHP, v0[k * HL + j], v1[k * HL + j], o0, o1);
+            for (int q = 0; q < BH; ++q) o[r][q] = 0.0f;
 #pragma unroll
-          for (int q = 0; q < BH; ++q) {
-            v0[q * HL + j] = o0[q];
-            v1[q * HL + j] = o1[q];
+          for (int k = 0; k < BH; ++k) {
+            float in[RPL];
+#pragma unroll
+            for (int r = 0; r < RPL; ++r) in[r] = v[r][k * HL + j];
+            axpy_bf<BH, RPL>(b + k * SB::BHP, in, o);
           }
+#pragma unroll
+          for (int r = 0; r < RPL; ++r)
+#pragma unroll
+            for (int q = 0; q < BH; ++q) v[r][q * HL + j] = o[r][q];
         }
       };
       auto stage_l = [&]() {
 #pragma unroll
         for (int iH = 0; iH < BH; ++iH) {
-          float o0[HL], o1[HL];
+          float o[RPL][HL];
 #pragma unroll
-          for (int q = 0; q < HL; ++q) o0[q] = o1[q] = 0.0f;
+          for (int r = 0; r < RPL; ++r)
+#pragma unroll
+            for (int q = 0; q < HL; ++q) o[r][q] = 0.0f;
           // outputs 2 q + h of block iH (contiguous after the column
           // permutation); inputs 2 j + h (own) and 2 j + 1 - h (partner)
-          const float* b = bl + SB::HF + iH * BL * SB::BLP + h * HL;
+          const uint16_t* b = bl + SB::HF + iH * BL * SB::BLP + h * HL;
 #pragma unroll
           for (int j = 0; j < HL; ++j) {
-            const float own0 = v0[iH * HL + j], own1 = v1[iH * HL + j];
-            const float oth0 = __shfl_xor_sync(0xffffffffu, own0, 16);
-            const float oth1 = __shfl_xor_sync(0xffffffffu, own1, 16);
-            axpy2<HL>(b + (2 * j + h) * SB::BLP, own0, own1, o0, o1);
-            axpy2<HL>(b + (2 * j + 1 - h) * SB::BLP, oth0, oth1, o0, o1);
+            float own[RPL], oth[RPL];
+#pragma unroll
+            for (int r = 0; r < RPL; ++r) {
+              own[r] = v[r][iH * HL + j];
+              oth[r] = __shfl_xor_sync(0xffffffffu, own[r], 16);
+            }
+            axpy_bf<HL, RPL>(b + (2 * j + h) * SB::BLP, own, o);
+            axpy_bf<HL, RPL>(b + (2 * j + 1 - h) * SB::BLP, oth, o);
           }
 #pragma unroll
-          for (int q = 0; q < HL; ++q) {
-            v0[iH * HL + q] = o0[q];
-            v1[iH * HL + q] = o1[q];
-          }
+          for (int r = 0; r < RPL; ++r)
+#pragma unroll
+            for (int q = 0; q < HL; ++q) v[r][iH * HL + q] = o[r][q];
         }
       };
       if (a.h_first) {
@@ -298,13 +315,12 @@ __global__ void __launch_bounds__(8 * R, 1)
         stage_h();
       }
 #pragma unroll
-      for (int iH = 0; iH < BH; ++iH)
+      for (int r = 0; r < RPL; ++r)
 #pragma unroll
-        for (int j = 0; j < HL; ++j) {
-          const int p = iH * BL + 2 * j + h;
-          st_elem<Tout>(s_out + box_offset<P, EO>(row0, p, lo), v0[iH * HL + j]);
-          st_elem<Tout>(s_out + box_offset<P, EO>(row0 + 1, p, lo), v1[iH * HL + j]);
-        }
+        for (int iH = 0; iH < BH; ++iH)
+#pragma unroll
+          for (int j = 0; j < HL; ++j)
+            st_elem<Tout>(s_out + box_offset<P, EO>(row0 + r, iH * BL + 2 * j + h, lo), v[r][iH * HL + j]);
       __syncthreads();
       // 16-byte global stores: piece (row, p) = the 8 lo values of one position
       constexpr int WO = 8 * EO / 16;  // 16-byte words per piece
@@ -321,12 +337,13 @@ __global__ void __launch_bounds__(8 * R, 1)
   }
 }
 
-template <int BH, int BL, int R, typename Tout>
+template <int BH, int BL, int RPL, typename Tout>
 cudaError_t launch_strided_t(const StridedArgs& a, cudaStream_t st) {
-  using G = StridedGeom<BH, BL, R, Tout>;
+  using G = StridedGeom<BH, BL, RPL, Tout>;
+  constexpr int R = G::R;
   static_assert(G::SMEM <= 227 * 1024, "shared memory");
   static std::atomic<unsigned long long> done{0};
-  auto kern = k_bfly_strided<BH, BL, R, Tout>;
+  auto kern = k_bfly_strided<BH, BL, RPL, Tout>;
   cudaError_t e = set_smem_attr(kern, G::SMEM, done);
   if (e != cudaSuccess) return e;
   int dev = 0, sms = 0;
@@ -358,9 +375,10 @@ cudaError_t launch_strided_t(const StridedArgs& a, cudaStream_t st) {
 
 template <int BH, int BL>
 cudaError_t launch_strided_b(int dt_out, const StridedArgs& a, cudaStream_t st) {
-  // 32-row boxes for bf16 results, 16-row boxes for fp32 (shared-memory budget)
-  return dt_out == DT_BF16 ? launch_strided_t<BH, BL, 32, __nv_bfloat16>(a, st)
-                           : launch_strided_t<BH, BL, 16, float>(a, st);
+  // two rows per lane (32-row boxes); three ran slower (the vectors and
+  // accumulators of three rows exceed the registers)
+  return dt_out == DT_BF16 ? launch_strided_t<BH, BL, 2, __nv_bfloat16>(a, st)
+                           : launch_strided_t<BH, BL, 2, float>(a, st);
 }
 
 }  // namespace
