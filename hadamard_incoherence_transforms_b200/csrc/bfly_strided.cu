@@ -384,8 +384,9 @@ cudaError_t launch_strided_t(const StridedArgs& a, cudaStream_t st) {
 // the first stage are, pairwise rounded to bf16, the A operands of the second
 // (the column order of one product is the row order of the next).  Only the
 // nonzero N tiles of each K step are issued: for M_H all BH of them (one
-// nonzero per eight lanes, read from shared memory per MMA), for M_L the two
-// of its own diagonal block (dense, two registers per lane read per MMA).
+// nonzero per eight lanes, read from shared memory per MMA, and only the K
+// half that holds them: m16n8k8), for M_L the two of its own diagonal block
+// (dense, two registers per lane read per MMA).
 // The A operands of the first stage come from the TMA box: the 32-bit word of
 // the warp's lo pair in each (row, position) row of 8 lo values.  Results go
 // to a shared-memory tile laid out per lo pair ([row][pair][position] words,
@@ -431,6 +432,13 @@ __device__ __forceinline__ void stage_blocks_ak(uint16_t* s_blk, int per_lo, int
   }
 }
 
+// m16n8k8: A = {a0, a1} (rows g, g + 8; k = 2 t, 2 t + 1), B = b0
+__device__ __forceinline__ void mma_1688(float (&d)[4], uint32_t a0, uint32_t a1, uint32_t b0) {
+  asm volatile(
+      "mma.sync.aligned.m16n8k8.row.col.f32.bf16.bf16.f32 {%0, %1, %2, %3}, {%4, %5}, {%6}, {%0, %1, %2, %3};"
+      : "+f"(d[0]), "+f"(d[1]), "+f"(d[2]), "+f"(d[3])
+      : "r"(a0), "r"(a1), "r"(b0));
+}
 __device__ __forceinline__ void mma_16816(float (&d)[4], uint32_t a0, uint32_t a1, uint32_t a2, uint32_t a3,
                                           uint32_t b0, uint32_t b1) {
   asm volatile(
@@ -561,9 +569,11 @@ __global__ void __launch_bounds__(256, 1)
             for (int aa = 0; aa < BH; ++aa) {
 #pragma unroll
               for (int hh = 0; hh < 2; ++hh) {
+                // the tile's nonzeros lie in K half hh: one m16n8k8 on that half
                 const uint32_t c = bh[(g + 8 * hh) * (BH * 8) + aa * 8 + j];
                 const uint32_t w = hact ? (c << hsh) : 0u;
-                mma_16816(acc[2 * aa + hh], a0, a1, a2, a3, hh ? 0u : w, hh ? w : 0u);
+                if (hh == 0) mma_1688(acc[2 * aa], a0, a1, w);
+                else mma_1688(acc[2 * aa + 1], a2, a3, w);
               }
             }
           }
