@@ -114,30 +114,43 @@ class ClockSampler:
     def _run(self):
         while not self._stop.is_set():
             try:
-                self.samples.append(self.nv.nvmlDeviceGetClockInfo(self.h, self.nv.NVML_CLOCK_SM))
+                mhz = self.nv.nvmlDeviceGetClockInfo(self.h, self.nv.NVML_CLOCK_SM)
                 r = self.nv.nvmlDeviceGetCurrentClocksEventReasons(self.h)
-                for bit, name in self.REASONS.items():
-                    if r & bit and name != "gpu_idle":
-                        self.reasons.add(name)
+                self.samples.append((time.perf_counter(), mhz, r))
             except Exception:
                 pass
-            time.sleep(0.001)  # the headline's timed region is only ~8 ms long
+            time.sleep(0.0002)  # the headline's timed region is only ~8 ms long
 
     def __enter__(self):
+        self.t_begin = time.perf_counter()
         if self.nv is not None:
             self.t = threading.Thread(target=self._run, daemon=True)
             self.t.start()
+            # the sampler is running before the timed region starts
+            t0 = time.perf_counter()
+            while len(self.samples) < 2 and time.perf_counter() - t0 < 0.5:
+                time.sleep(0.0005)
+        self.t_begin = time.perf_counter()
         return self
 
     def __exit__(self, *exc):
+        self.t_end = time.perf_counter()
         self._stop.set()
         if self.nv is not None:
             self.t.join()
 
     def summary(self):
-        med = statistics.median(self.samples) if self.samples else None
-        return {"sm_mhz": med, "sm_max_mhz": self.max_mhz, "reasons": sorted(self.reasons),
-                "samples": len(self.samples)}
+        """Samples taken while the timed region ran (host window around it);
+        the last earlier sample if none fell inside."""
+        inside = [s for s in self.samples if self.t_begin <= s[0] <= getattr(self, "t_end", float("inf"))]
+        used = inside or self.samples[-1:]
+        reasons = set()
+        for _, _, r in used:
+            for bit, name in self.REASONS.items():
+                if r & bit and name != "gpu_idle":
+                    reasons.add(name)
+        med = statistics.median(m for _, m, _ in used) if used else None
+        return {"sm_mhz": med, "sm_max_mhz": self.max_mhz, "reasons": sorted(reasons), "samples": len(inside)}
 
 
 def read_profile_traffic(kernel_key: str):
