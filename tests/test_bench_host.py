@@ -113,3 +113,33 @@ def test_clock_sampler_without_nvml(monkeypatch):
     with bench.ClockSampler(0) as clk:
         pass
     assert clk.summary() == {"sm_mhz": None, "sm_max_mhz": None, "reasons": [], "samples": 0}
+
+
+def test_clock_sampler_reports_only_the_timed_window(monkeypatch):
+    """Samples taken while the sampler starts up (before the timed region)
+    are not part of the summary."""
+    import sys
+    import time
+    import types
+
+    state = {"n": 0}
+
+    def clock(h, kind):
+        state["n"] += 1
+        return 1000 if state["n"] <= 2 else 1965   # the start-up samples read 1000 MHz
+
+    fake = types.SimpleNamespace(
+        NVML_CLOCK_SM=1,
+        nvmlInit=lambda: None,
+        nvmlDeviceGetHandleByIndex=lambda i: ("h", i),
+        nvmlDeviceGetMaxClockInfo=lambda h, kind: 1965,
+        nvmlDeviceGetClockInfo=clock,
+        nvmlDeviceGetCurrentClocksEventReasons=lambda h: 0,
+    )
+    monkeypatch.setitem(sys.modules, "pynvml", fake)
+    monkeypatch.delenv("CUDA_VISIBLE_DEVICES", raising=False)
+    with bench.ClockSampler(0) as clk:
+        time.sleep(0.02)
+    out = clk.summary()
+    assert out["samples"] >= 3 and out["sm_mhz"] == 1965 and out["reasons"] == []
+    assert len(clk.samples) > out["samples"]   # the start-up samples were taken, then left out
