@@ -169,6 +169,11 @@ HIT_API int butterfly_apply(const void* x, void* y, int64_t rows, int64_t n, int
  *     (windows of 128 contiguous positions holding 128 / P groups);
  *   along columns (axis 0): digits with P in {128, 256} (positions at the
  *     stride of the run's last digit), or the last digits with P dividing 128;
+ * two adjacent digits along rows at a stride that is a multiple of 8, with
+ * radices (7, 16), (4, 16), (8, 8) or (16, 4), run as one register-resident
+ * pass with their blocks rounded to bf16: on mma.sync tensor-core tiles
+ * (block-diagonal products, bf16 between the two stages) for (7, 16) and
+ * (4, 16) with a bf16 result, else in fp32 SIMT arithmetic;
  * other runs use the SIMT passes of butterfly_apply.  Data between passes is
  * bf16, so results carry bf16 rounding per pass (use butterfly_apply for an
  * fp32-accurate rotation).
