@@ -226,7 +226,8 @@ def test_butterfly_tc_host_checks_and_workspace(lib):
         r = (ct.c_int32 * len(radices))(*radices)
         return lib.butterfly_tc_workspace_bytes(rows, n, axis, len(radices), ct.cast(r, ct.c_void_p), transpose)
 
-    # R_in of the butterfly workload: {2,3} on tensor cores (window 128), {0,1} SIMT, one bf16 intermediate
+    # R_in of the butterfly workload: {2,3} on tensor cores (window 128), {0,1} a strided two-digit run
+    # (no window matrix), one bf16 intermediate
     assert ws(4096, 14336, 1, (7, 16, 16, 8)) >= 14336 * 128 * 2 + 4096 * 14336 * 2
     # R_out: {0,1} (window 256 at stride 16) and {2} (block-diagonal windows of 128)
     assert ws(4096, 14336, 0, (16, 16, 16)) >= 4096 * 256 * 2 + 4096 * 128 * 2 + 4096 * 14336 * 2
